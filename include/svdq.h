@@ -1,0 +1,172 @@
+/*
+ * svdq.h -- C ABI of the SVDQuant W4A4 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer (SVDQuant; "SVDQuant是什么？" 技术原理, "AI图像生成4-bit量化技术解析与应用"
+ * 2.2/3.1/3.2, "DeepCompressor…" SVDQuant section):
+ *
+ *     X^ = X diag(lambda)^-1,  W^ = diag(lambda) W         smoothing
+ *     W^ ~ L1 L2  (rank r, truncated SVD, 16-bit)          low-rank branch
+ *     R  = W^ - L1 L2                                       4-bit residual
+ *     Y  = Q(X^) Q(R) + (X^ L1) L2 + b
+ *
+ * Q is INT4 with symmetric per-group-of-64 fp32 scales, or NVFP4 (E2M1 values,
+ * one E4M3 scale per 16 values, one fp32 tensor scale).
+ *
+ * Two halves:
+ *   svdq_prepare  host, offline: smoothing factors, truncated SVD, residual,
+ *                 weight quantisation, packing into one self-describing blob.
+ *   svdq_linear   device, per call: activation quantisation + down projection
+ *                 (one kernel), then the 4-bit GEMM whose epilogue adds the
+ *                 low-rank up projection and the bias (one kernel).
+ *
+ * Layout conventions (all row-major, C order):
+ *   Wt    N x K  fp32, nn.Linear layout (W = Wt^T is K x N); host memory.
+ *   X     M x K  fp16 or bf16 (params.act_dtype); device memory.
+ *   Y     M x N  bf16; device memory.
+ *   bias  N fp32 or NULL (zero bias); host memory.
+ *
+ * Ownership: the caller allocates and owns every buffer (host and device).
+ * The library allocates no device memory and keeps no per-call state; one
+ * device-global status word per GPU records device-side failures.
+ *
+ * Errors: every function returns an svdq_status and never aborts.  Device
+ * work is launched asynchronously; failures inside a kernel (a bounded wait
+ * that gave up) are recorded in the status word and read by svdq_get_status.
+ *
+ * Constraints: K % 128 == 0, N % 256 == 0, 0 <= rank <= 128, rank % 16 == 0,
+ * M >= 0 (M = 0 is a no-op), device pointers 16-byte aligned, inputs finite.
+ */
+#ifndef SVDQ_H
+#define SVDQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,    /* null pointer, bad size or unsupported shape   */
+  SVDQ_ERR_UNSUPPORTED = 2,    /* no sm_100 device or unsupported format         */
+  SVDQ_ERR_ALIGNMENT = 3,      /* a device pointer is not 16-byte aligned        */
+  SVDQ_ERR_WORKSPACE = 4,      /* workspace smaller than svdq_workspace_bytes    */
+  SVDQ_ERR_BLOB = 5,           /* blob header, size or checksum mismatch         */
+  SVDQ_ERR_NO_CONVERGENCE = 6, /* truncated SVD did not converge                 */
+  SVDQ_ERR_CUDA = 7,           /* a CUDA runtime call or launch failed           */
+  SVDQ_ERR_TIMEOUT = 8         /* a device-side bounded wait gave up             */
+} svdq_status;
+
+typedef enum { SVDQ_INT4_G64 = 1, SVDQ_NVFP4 = 2 } svdq_format;
+typedef enum { SVDQ_F16 = 1, SVDQ_BF16 = 2 } svdq_dtype;
+
+typedef struct svdq_params {
+  int32_t K;          /* input features                                   */
+  int32_t N;          /* output features                                  */
+  int32_t rank;       /* r, rank of the 16-bit branch (0 disables it)     */
+  int32_t fmt;        /* svdq_format                                      */
+  int32_t act_dtype;  /* svdq_dtype of X (and of the stored L1, L2)       */
+  int32_t smooth;     /* 1: smoothing on; 0: lambda = 1                   */
+  float alpha;        /* smoothing migration strength, in [0, 1]          */
+  int32_t reserved;   /* must be 0                                        */
+} svdq_params;
+
+/* An opaque CUDA stream handle (cudaStream_t); NULL is the legacy default stream. */
+typedef struct CUstream_st* svdq_stream;
+
+/* ---------------------------------------------------------------- host side */
+
+/* Bytes of the blob svdq_prepare writes for these parameters (0 if invalid). */
+size_t svdq_blob_bytes(const svdq_params* p);
+
+/*
+ * Offline preparation ("SVDQuant是什么？" 技术原理; 4-bit page 2.2).
+ *   lambda_j = a_j^alpha / w_j^(1-alpha), a_j = max_m |X_cal[m,j]|,
+ *   w_j = max_n |W[j,n]| (1 where either is 0 or smoothing is off);
+ *   W^ = diag(lambda) W; (L1, L2) = top-r singular triplets of W^ as
+ *   L1 = U_r S_r, L2 = V_r^T rounded to act_dtype; R = W^ - L1 L2 (float64,
+ *   then fp32); R quantised per output channel along K; NVFP4 also stores the
+ *   static activation tensor scale amax(X_cal diag(lambda)^-1) / 2688.
+ * Wt: N x K fp32 host.  bias: N fp32 host or NULL.  X_cal: M_cal x K host,
+ * act_dtype bits (calibration activations; may be the layer's own input).
+ * blob: host buffer of blob_bytes >= svdq_blob_bytes(p); copy it to device
+ * memory (16-byte aligned) before svdq_linear.  sigma_out: NULL or rank+1
+ * doubles, the leading singular values of W^ (estimates).
+ * Uses the host's cores (OpenMP).  Deterministic for a given input.
+ */
+svdq_status svdq_prepare(const svdq_params* p, const float* Wt, const float* bias,
+                         const void* X_cal, int64_t M_cal, void* blob, size_t blob_bytes,
+                         double* sigma_out);
+
+/* Validate a host blob against p: magic, version, parameters, size, checksum. */
+svdq_status svdq_blob_check(const svdq_params* p, const void* blob, size_t blob_bytes);
+
+/*
+ * Copy a host blob's contents out in a canonical, layout-independent form
+ * (for tests and inspection).  Any output pointer may be NULL.
+ *   inv_lambda  K fp32
+ *   L1          K x r  act_dtype bits (uint16)
+ *   L2          r x N  act_dtype bits (uint16)
+ *   wcodes      N x K  one code per byte: INT4 as int8 in [-8, 7];
+ *               NVFP4 as the E2M1 code in the low nibble
+ *   wscales     INT4: N x K/64 fp32;  NVFP4: N x K/16 E4M3 codes (uint8)
+ *   tscales     2 fp32: [s_gX, s_gW] (NVFP4 tensor scales; 1 for INT4)
+ *   bias        N fp32
+ */
+svdq_status svdq_blob_export(const svdq_params* p, const void* blob, float* inv_lambda,
+                             uint16_t* L1, uint16_t* L2, uint8_t* wcodes, void* wscales,
+                             float* tscales, float* bias);
+
+/* Device workspace bytes svdq_linear needs for M tokens. */
+size_t svdq_workspace_bytes(const svdq_params* p, int64_t M);
+
+/* ---------------------------------------------------------------- device side */
+
+/*
+ * Y = Q(X^) Q(R) + (X^ L1) L2 + b for M tokens ("DeepCompressor…" SVDQuant
+ * section: the low-rank branch is fused into the low-bit kernel).
+ *   Kernel 1 reads X once: X^ = fp32(X) * inv_lambda, per-token dynamic
+ *   quantisation (INT4 groups of 64 / NVFP4 blocks of 16 with the static
+ *   tensor scale) and u = X^16 L1 (X^ rounded to act_dtype, fp32 accumulate).
+ *   Kernel 2: TMA-fed tcgen05 GEMM with TMEM accumulators; the epilogue adds
+ *   u L2 (as extra tensor-core K-steps into the same accumulator) and b, and
+ *   writes bf16 Y.
+ * blob_dev: device copy of the svdq_prepare blob for the same p.
+ * X: M x K act_dtype, device.  Y: M x N bf16, device.
+ * workspace: device, >= svdq_workspace_bytes(p, M); holds the quantised
+ * activations between the kernels (read back by svdq_export_act).
+ * Asynchronous on `stream`; returns SVDQ_ERR_CUDA if a launch fails.
+ */
+svdq_status svdq_linear(const svdq_params* p, const void* blob_dev, const void* X, int64_t M,
+                        void* Y, void* workspace, size_t ws_bytes, svdq_stream stream);
+
+/*
+ * After svdq_linear: copy the quantised activations out of the workspace in
+ * canonical form (synchronises `stream`).  Any output pointer may be NULL.
+ *   codes   M x K host, one code per byte (INT4 int8 / NVFP4 E2M1 low nibble)
+ *   scales  INT4: M x K/64 fp32;  NVFP4: M x K/16 E4M3 codes (uint8)
+ *   u       M x r host fp32: the down projection X^16 L1 as used by kernel 2
+ *           (hi + lo parts summed, before the tensor-scale division)
+ */
+svdq_status svdq_export_act(const svdq_params* p, const void* workspace, int64_t M,
+                            uint8_t* codes, void* scales, float* u, svdq_stream stream);
+
+/* Synchronise `stream`, read and clear this device's status word. */
+svdq_status svdq_get_status(svdq_stream stream);
+
+const char* svdq_status_string(svdq_status s);
+
+/*
+ * Test hook: the GPU's own fp32 -> E2M1 and fp32 -> E4M3 conversions
+ * (cvt.rn.satfinite), used to pin the host encoders.  in: n fp32 device;
+ * e2m1, e4m3: n bytes device (one code per byte).  Asynchronous.
+ */
+svdq_status svdq_probe_cvt(const float* in, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
+                           svdq_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H */

@@ -1,0 +1,117 @@
+// Internal layouts of the blob (prepared weights) and of the per-call workspace.
+//
+// Blob (one contiguous buffer, every section 1024-byte aligned):
+//   header      BlobHeader
+//   inv_lambda  K fp32                                  smoothing, device multiplies X by it
+//   l1t         r x K act_dtype (L1 transposed)          B operand of the down projection
+//   l2x         N x lrw bf16, K-major                    B operand of the up projection
+//               (lrw = nseg*r rounded up to 64, zero padded):
+//               bf16 X: [L2 ; L2]             (pairs with [u_hi | u_lo])
+//               fp16 X: [L2h ; L2h ; L2l]     (pairs with [u_hi | u_lo | u_hi]; L2 = L2h + L2l exactly)
+//   wq          NVFP4: N x K/2 bytes, E2M1 packed, element k in the low nibble when k is even
+//               INT4:  N x K bytes, the code as an E4M3 byte (exact for -8..7)
+//   ws          NVFP4: E4M3 block scales in the tcgen05 scale-factor atom layout (below)
+//               INT4:  fp32 [K/64][N]
+//   bias        N fp32
+//
+// Workspace for M tokens:
+//   xq   NVFP4: M x K/2 bytes packed E2M1;   INT4: M x K bytes (code as E4M3 byte)
+//   xs   NVFP4: scale-factor atoms for ceil(M/128)*128 rows;  INT4: fp32 [K/64][Mp], Mp = ceil(M/128)*128
+//   ux   M x lrw bf16: [u'_hi | u'_lo (| u'_hi) | 0 pad], u' = u / (s_gX s_gW) (NVFP4) or u (INT4)
+//
+// Scale-factor atom layout (the operand format of tcgen05 block-scaled MMA
+// scale factors once copied to tensor memory by tcgen05.cp 32x128b.warpx4):
+// rows are grouped by 128, scale blocks along K by 4 (64 elements); each group
+// is a 512-byte atom, atoms ordered [row_group][k_group]; inside an atom the
+// scale of row r (0..127) and block j (0..3) sits at byte (r%32)*16 + (r/32)*4 + j.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/svdq.h"
+
+namespace svdq {
+
+constexpr uint32_t kMagic0 = 0x51445653u;  // "SVDQ"
+constexpr uint32_t kMagic1 = 0x30303242u;  // "B200"
+constexpr uint32_t kVersion = 1;
+constexpr size_t kAlign = 1024;
+constexpr int kGroupInt4 = 64;
+constexpr int kBlockFp4 = 16;
+
+struct BlobHeader {
+  uint32_t magic0, magic1, version, header_bytes;
+  svdq_params params;
+  uint64_t total_bytes;
+  uint64_t off_inv_lambda, off_l1t, off_l2x, off_wq, off_ws, off_bias;
+  float s_gx, s_gw;
+  int32_t nseg, pad0;
+  uint64_t checksum;  // FNV-1a 64 over bytes [header_bytes, total_bytes)
+};
+static_assert(sizeof(BlobHeader) <= kAlign, "header too large");
+
+inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+
+#ifdef __CUDACC__
+#define SVDQ_HD __host__ __device__
+#else
+#define SVDQ_HD
+#endif
+
+inline int nseg_of(const svdq_params& p) { return p.act_dtype == SVDQ_F16 ? 3 : 2; }
+// Width (bf16 elements) of one row of the low-rank operands.
+inline int lr_width(const svdq_params& p) { return (nseg_of(p) * p.rank + 63) / 64 * 64; }
+
+struct BlobLayout {
+  size_t off_inv_lambda, off_l1t, off_l2x, off_wq, off_ws, off_bias, total;
+  int nseg;
+};
+
+inline BlobLayout blob_layout(const svdq_params& p) {
+  BlobLayout L{};
+  const size_t K = (size_t)p.K, N = (size_t)p.N, r = (size_t)p.rank;
+  L.nseg = nseg_of(p);
+  size_t off = kAlign;
+  L.off_inv_lambda = off; off = align_up(off + K * 4);
+  L.off_l1t = off;        off = align_up(off + r * K * 2);
+  L.off_l2x = off;        off = align_up(off + N * (size_t)lr_width(p) * 2);
+  L.off_wq = off;
+  off = align_up(off + (p.fmt == SVDQ_NVFP4 ? N * K / 2 : N * K));
+  L.off_ws = off;
+  off = align_up(off + (p.fmt == SVDQ_NVFP4 ? N * (K / kBlockFp4) : (K / kGroupInt4) * N * 4));
+  L.off_bias = off;       off = align_up(off + N * 4);
+  L.total = off;
+  return L;
+}
+
+struct WsLayout {
+  size_t off_xq, off_xs, off_ux, total;
+  int64_t Mp;  // M rounded up to 128
+};
+
+inline WsLayout ws_layout(const svdq_params& p, int64_t M) {
+  WsLayout L{};
+  const size_t K = (size_t)p.K;
+  L.Mp = (M + 127) / 128 * 128;
+  const size_t Mp = (size_t)L.Mp;
+  size_t off = 0;
+  L.off_xq = off;
+  off = align_up(off + (p.fmt == SVDQ_NVFP4 ? (size_t)M * K / 2 : (size_t)M * K));
+  L.off_xs = off;
+  off = align_up(off + (p.fmt == SVDQ_NVFP4 ? Mp * (K / kBlockFp4) : (K / kGroupInt4) * Mp * 4));
+  L.off_ux = off;
+  off = align_up(off + (size_t)M * (size_t)lr_width(p) * 2);
+  L.total = off > 0 ? off : kAlign;
+  return L;
+}
+
+// Byte offset of scale (row, block) inside a scale-factor atom array whose
+// rows span `kblocks` blocks of 16 along K (kblocks % 4 == 0).
+SVDQ_HD inline size_t sf_offset(int64_t row, int64_t blk, int64_t kblocks) {
+  const int64_t atom = (row / 128) * (kblocks / 4) + blk / 4;
+  const int64_t r = row % 128;
+  return (size_t)(atom * 512 + (r % 32) * 16 + (r / 32) * 4 + (blk % 4));
+}
+
+}  // namespace svdq

@@ -1,0 +1,108 @@
+"""svdq_linear on the GPU against the CPU oracle, through the C ABI.
+
+Bit-exact: activation codes and scales (and, via the host prepare, weight
+codes and scales).  Y: relative Frobenius error <= 1e-3 against the oracle's
+output rounded to bf16.  Guard rows around Y and a guard tail behind the
+workspace catch out-of-bounds writes.
+"""
+import numpy as np
+import pytest
+
+import rank_gemm_svdq_b200 as sv
+import synth
+from oracle import formats
+from tests import gpu_cases as G
+
+pytestmark = pytest.mark.gpu
+
+
+def test_probe_cvt_matches_oracle_encoders(gpu):
+    """The GPU's cvt.rn.satfinite to E2M1 / E4M3 equals the oracle's
+    round-to-nearest-even encoders (ties, saturation, signed zero)."""
+    import torch
+    rng = np.random.default_rng(1)
+    e2 = formats.E2M1_VALUES[:8]; e4 = formats.E4M3_VALUES[:0x7F]
+    mids = np.concatenate([0.5 * (e2[:-1] + e2[1:]), 0.5 * (e4[:-1] + e4[1:])]).astype(np.float32)
+    x = np.concatenate([mids, np.nextafter(mids, np.float32(np.inf)), np.nextafter(mids, np.float32(0)),
+                        e2.astype(np.float32), e4.astype(np.float32),
+                        rng.uniform(0, 8, 20000).astype(np.float32),
+                        np.exp(rng.uniform(-14, 7, 20000)).astype(np.float32),
+                        np.array([1e-30, 1e30, 500.0, 464.0, 6.5, 7.0, 0.0], np.float32)])
+    x = np.concatenate([x, -x])
+    xd = torch.from_numpy(x).cuda()
+    o2 = torch.zeros(len(x), dtype=torch.uint8, device="cuda")
+    o4 = torch.zeros(len(x), dtype=torch.uint8, device="cuda")
+    sv.probe_cvt(xd, o2, o4)
+    torch.cuda.synchronize()
+    g2, g4 = o2.cpu().numpy(), o4.cpu().numpy()
+    r2 = formats.e2m1_encode(x.astype(np.float64)); r4 = formats.e4m3_encode(x.astype(np.float64))
+    bad2 = np.flatnonzero(g2 != r2); bad4 = np.flatnonzero(g4 != r4)
+    assert len(bad2) == 0, (x[bad2[:8]], g2[bad2[:8]], r2[bad2[:8]])
+    assert len(bad4) == 0, (x[bad4[:8]], g4[bad4[:8]], r4[bad4[:8]])
+
+
+def test_tiny_int4_config(gpu):
+    """The tiny INT4 layer (M=256, K=512, N=512, fp16, rank 16, 4 outlier
+    channels x100): every output and every code against the oracle."""
+    pp = G.prepared_preset("tiny_int4")
+    run = G.run_gpu(pp, pp.wl.X)
+    G.compare(pp, pp.wl.X, run)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("M,rank", [(1, 16), (127, 32), (129, 0), (300, 16), (384, 48)])
+def test_small_shapes(gpu, fmt, dtype, M, rank):
+    """Ragged token counts (1, 127, 129, 300: partial 128-row tiles), several
+    tiles along N and K, rank 0 (no low-rank branch) and rank 48 (two
+    low-rank K-steps for fp16)."""
+    wl = synth.custom_workload(M, 512, 768, rank, fmt, dtype, n_out=5, factor=80.0, seed=M + rank)
+    pp = G.prepare(wl)
+    run = G.run_gpu(pp, wl.X)
+    G.compare(pp, wl.X, run)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+def test_zero_input_gives_bias(gpu, fmt):
+    wl = synth.custom_workload(64, 256, 512, 16, fmt, "bf16", n_out=2, factor=10.0, seed=5)
+    pp = G.prepare(wl)
+    X0 = np.zeros_like(wl.X)
+    run = G.run_gpu(pp, X0)
+    assert np.all(run.codes.view(np.uint8) == 0)
+    assert np.array_equal(run.Y, np.broadcast_to(formats.to_bf16(wl.bias.astype(np.float64)), run.Y.shape))
+
+
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+def test_repeat_calls_are_bitwise_identical(gpu, fmt):
+    wl = synth.custom_workload(200, 512, 512, 32, fmt, "bf16", n_out=4, factor=50.0, seed=9)
+    pp = G.prepare(wl)
+    a = G.run_gpu(pp, wl.X)
+    b = G.run_gpu(pp, wl.X)
+    assert np.array_equal(a.Y, b.Y) and np.array_equal(a.codes, b.codes)
+
+
+@pytest.mark.parametrize("name", ["flux_qkv_int4", "flux_ffn_up_nvfp4", "ffn_down_nvfp4", "ffn_down_int4"])
+def test_full_size_config(gpu, name):
+    """Full-size FLUX / FFN-down layers in the benchmark's launch configuration:
+    codes on 512 sampled tokens and Y on ~100 sampled tokens (incl. tile edges)."""
+    pp = G.prepared_preset(name)
+    X = pp.wl.X
+    run = G.run_gpu(pp, X)
+    M = X.shape[0]
+    res = G.compare(pp, X, run, rows=G.sample_rows(M), code_rows=G.sample_rows(M, 500, seed=1))
+    print(name, res)
+
+
+@pytest.mark.parametrize("shape", ["var_up_nvfp4", "var_down_nvfp4"])
+def test_var_token_sweep(gpu, shape):
+    """Infinity-VAR style projections at every token count of the sweep."""
+    pp = G.prepared_preset(shape)
+    for M in synth.VAR_TOKENS:
+        X = pp.wl.X[:M]
+        run = G.run_gpu(pp, X)
+        rows = G.sample_rows(M, 48)
+        G.compare(pp, X, run, rows=rows, code_rows=rows)
+
+
+def test_status_word_clean(gpu):
+    assert sv.get_status() == sv.OK

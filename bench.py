@@ -1,0 +1,371 @@
+#!/usr/bin/env python
+"""Benchmark of the SVDQuant W4A4 linear layer (svdq_linear) on B200.
+
+Workload: FLUX.1-like FFN up projection, M=4608 tokens (4096 image + 512
+text), K=3072, N=12288, rank 32, NVFP4 (E2M1 + E4M3 per 16 + fp32 tensor
+scale), bf16 activations with 1% outlier channels x50 -- synthetic data of
+that shape (no trained weights or activations exist here).
+
+One step = one svdq_linear call (activation quantisation + down projection
+kernel, then the tcgen05 GEMM with the fused low-rank epilogue) over one batch
+of 4608 tokens resident in HBM.  L2 is flushed (256 MiB write) before every
+timed step; each step is timed with CUDA events on the launching stream.
+
+Metric: TFLOP/s = (2 M K N + 2 M r (K + N)) / t.  Multi-GPU (torchrun): one
+independent layer replica per GPU, each with its own token batch (weak
+scaling, no data-path collective); value = all ranks' FLOPs / max-over-ranks
+time.  `--impl reference` times the CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "flux_ffn_up_nvfp4"
+METRIC = "fused SVDQuant W4A4 linear TFLOP/s and % of B200 FP4/INT8 tensor peak"
+NOMINAL_FP4_TFLOPS = 9000.0
+NOMINAL_BF16_TFLOPS = 2250.0
+FLUSH_BYTES = 256 << 20
+
+
+def flops(M, K, N, r):
+    return 2.0 * M * K * N + 2.0 * M * r * (K + N)
+
+
+def gemm_alg_bytes(M, K, N, r, fmt):
+    """Algorithmic bytes of one GEMM launch (kernel 2): quantised X codes and
+    scales + the down projection in, weight codes/scales + L2 + bias in,
+    bf16 Y out."""
+    xq = M * K // 2 + M * K // 16 if fmt == "nvfp4" else M * K + M * (K // 64) * 4
+    wq = N * K // 2 + N * K // 16 if fmt == "nvfp4" else N * K + N * (K // 64) * 4
+    return xq + M * 2 * r * 2 + wq + N * 2 * r * 2 + N * 4 + M * N * 2
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 50 ms in a thread."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_id: str):
+        self.dev_id = dev_id
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
+                 "-i", self.dev_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        rows = [s for (t, s) in self.samples if t0 - 0.06 <= t <= t1 + 0.06] or \
+               [s for (_, s) in self.samples]
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0])); mx = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def device_smi_id(torch, dev):
+    try:
+        pr = torch.cuda.get_device_properties(dev)
+        return f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        return vis.split(",")[dev] if vis else str(dev)
+
+
+def oracle_layer(wl):
+    """The CPU oracle's layer, built from the library's host-prepared factors
+    (the offline SVD is not part of the timed linear)."""
+    import rank_gemm_svdq_b200 as sv
+    import synth
+    from oracle import svdquant as sq
+    p = sv.params(wl.K, wl.N, wl.rank, wl.fmt, wl.dtype, wl.alpha, wl.smooth)
+    blob, _ = sv.prepare(p, wl.Wt, wl.bias, wl.X)
+    c = sv.blob_export(p, blob)
+    L1, L2 = synth.bf16_bits_to_f64(c.L1), synth.bf16_bits_to_f64(c.L2)
+    return sq.prepare(wl.x_f64(), wl.Wt, wl.bias, wl.rank, wl.fmt, wl.dtype, wl.alpha, wl.smooth,
+                      factors=(c.inv_lambda, L1, L2))
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max(i["num_threads"] for i in threadpool_info())
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(wl, ref, min_seconds=10.0):
+    """The oracle's linear part over the whole layer (all M tokens), repeated
+    until at least `min_seconds` of CPU work."""
+    from oracle import svdquant as sq
+    x = wl.x_f64()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        sq.forward(x, ref)
+        reps += 1
+        if time.perf_counter() - t0 >= min_seconds:
+            break
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": flops(wl.M, wl.K, wl.N, wl.rank) / dt / 1e12, "unit": "TFLOP/s",
+            "cores": blas_threads(), "kind": "oracle",
+            "sample": f"whole layer ({wl.M} tokens) x {reps} repetitions, {dt:.2f} s each, float64 numpy/BLAS"}
+
+
+def config_dict(wl, extra=None):
+    d = {"workload": f"{WORKLOAD}: FLUX.1-like FFN up projection M={wl.M} K={wl.K} N={wl.N} rank={wl.rank} "
+                     f"NVFP4 (E2M1, E4M3/16, fp32 tensor scale), bf16 X, 1% outlier channels x50",
+         "M": wl.M, "K": wl.K, "N": wl.N, "rank": wl.rank, "format": "nvfp4", "act_dtype": "bf16",
+         "l2": "flushed by a 256 MiB write before every timed step"}
+    if extra:
+        d.update(extra)
+    return d
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import synth
+    wl = synth.make_workload(WORKLOAD)
+    ref = oracle_layer(wl)
+    from oracle import svdquant as sq
+    x = wl.x_f64()
+    S = 256
+    times = []
+    for it in range(args.warmup + args.steps):
+        rows = slice((it * S) % wl.M, (it * S) % wl.M + S)
+        t0 = time.perf_counter()
+        sq.forward(x[rows], ref)
+        dt = time.perf_counter() - t0
+        if it >= args.warmup:
+            times.append(dt)
+    tot = sum(times)
+    value = flops(S, wl.K, wl.N, wl.rank) * len(times) / tot / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(wl, {"sample_tokens_per_step": S}),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{S} of the {wl.M} tokens per step (oracle float64, numpy/BLAS)"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import rank_gemm_svdq_b200 as sv
+    import synth
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    wl = synth.make_workload(WORKLOAD, seed=0)
+    if rank > 0:   # each replica gets its own token batch (same layer)
+        info = {}
+        wl.X = synth.make_x(rank, wl.M, wl.K, wl.dtype, 31, 50.0, info=info)
+    p = sv.params(wl.K, wl.N, wl.rank, wl.fmt, wl.dtype, wl.alpha, wl.smooth)
+    blob_host, _ = sv.prepare(p, wl.Wt, wl.bias, wl.X)
+    dev = torch.device("cuda", local)
+    blob = torch.from_numpy(blob_host).to(dev)
+    X = torch.from_numpy(wl.X.view(np.int16)).to(dev).view(torch.bfloat16)
+    Y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(sv.workspace_bytes(p, wl.M), dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    M, K, N, r = wl.M, wl.K, wl.N, wl.rank
+
+    def timed(fn, steps):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            evs[i][0].record(stream)
+            fn()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in evs]
+
+    def step():
+        sv.linear(p, blob, X, M, Y, ws, stream)
+
+    # warm-up
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize()
+    assert sv.get_status() == sv.OK
+
+    sampler = ClockSampler(device_smi_id(torch, local))
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    ms = timed(step, args.steps)
+    torch.cuda.synchronize()
+    barrier()
+    t1 = time.time()
+    time.sleep(0.1)
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
+    st = sv.get_status()
+    assert st == sv.OK, sv.status_string(st)
+
+    total_ms = float(sum(ms))
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = flops(M, K, N, r) * world / (ms_per_step * 1e-3) / 1e12
+
+    # per-kernel timing (same flushes), for the roofline of the dominant kernel
+    def quant_only():
+        sv.quantize_act(p, blob, X, M, ws, stream)
+
+    def gemm_only():
+        sv.gemm(p, blob, M, Y, ws, stream)
+
+    ksteps = min(args.steps, 100)
+    ms_act = float(np.mean(timed(quant_only, ksteps)))
+    quant_only()
+    ms_gemm = float(np.mean(timed(gemm_only, ksteps)))
+
+    # end to end through the C ABI with host buffers: pinned X in, Y out
+    Xh = torch.from_numpy(wl.X.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    Xd = torch.empty_like(X)
+
+    def e2e_step():
+        Xd.copy_(Xh, non_blocking=True)
+        sv.linear(p, blob, Xd, M, Y, ws, stream)
+        Yh.copy_(Y, non_blocking=True)
+
+    esteps = min(args.steps, 50)
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e_ms = timed(e2e_step, esteps)
+    e_total = float(sum(e_ms))
+    if dist is not None:
+        t = torch.tensor([e_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_total = float(t.item())
+    e2e_value = flops(M, K, N, r) * world / (e_total / esteps * 1e-3) / 1e12
+    assert sv.get_status() == sv.OK
+
+    peaks = measured_peaks()
+    if peaks and "bf16_tflops_sustained" in peaks:
+        peak = float(peaks["bf16_tflops_sustained"]) * (NOMINAL_FP4_TFLOPS / NOMINAL_BF16_TFLOPS)
+        peak_note = ("of measured: sustained cuBLAS bf16 "
+                     f"{peaks['bf16_tflops_sustained']} TFLOP/s x 4 (nominal dense FP4/BF16 ratio)")
+    else:
+        peak = 1400.0 * 4
+        peak_note = "of fallback: 1.4 PFLOP/s sustained bf16 x 4"
+    gemm_flops = flops(M, K, N, r)
+    achieved = gemm_flops / (ms_gemm * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "gemm_nvfp4_kernel", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None, "peak_source": peak_note,
+                "frac_of_nominal_fp4": achieved / NOMINAL_FP4_TFLOPS,
+                "alg_flops_per_launch": gemm_flops,
+                "alg_bytes_per_launch": gemm_alg_bytes(M, K, N, r, "nvfp4"),
+                "kernel_ms": {"gemm": ms_gemm, "act_quant": ms_act}}
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+            "config": config_dict(wl, {"parallelism": f"replicas x{world} (token batches, no collective)"}),
+            "roofline": roofline, "clocks": clocks, "gpu_launches": 2 * args.steps,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(X.numel() * 2),
+                    "d2h_bytes_per_step": int(Y.numel() * 2)},
+            "frac_of_nominal_fp4": value / NOMINAL_FP4_TFLOPS}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, oracle_layer(wl))
+    if dist is not None:
+        barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

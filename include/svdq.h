@@ -33,7 +33,8 @@
  * work is launched asynchronously; failures inside a kernel (a bounded wait
  * that gave up) are recorded in the status word and read by svdq_get_status.
  *
- * Constraints: K % 128 == 0, N % 256 == 0, 0 <= rank <= 128, rank % 16 == 0,
+ * Constraints: K % 128 == 0 (INT4) or K % 256 == 0 (NVFP4), N % 256 == 0,
+ * 0 <= rank <= 128, rank % 16 == 0,
  * M >= 0 (M = 0 is a no-op), device pointers 16-byte aligned, inputs finite.
  */
 #ifndef SVDQ_H
@@ -142,6 +143,17 @@ svdq_status svdq_linear(const svdq_params* p, const void* blob_dev, const void* 
                         void* Y, void* workspace, size_t ws_bytes, svdq_stream stream);
 
 /*
+ * The two halves of svdq_linear as separate launches (same arguments and
+ * rules).  svdq_quantize_act runs kernel 1 (X -> workspace); svdq_gemm runs
+ * kernel 2 (workspace -> Y) and must follow a svdq_quantize_act for the same
+ * M and workspace in stream order.  svdq_linear == quantize_act + gemm.
+ */
+svdq_status svdq_quantize_act(const svdq_params* p, const void* blob_dev, const void* X, int64_t M,
+                              void* workspace, size_t ws_bytes, svdq_stream stream);
+svdq_status svdq_gemm(const svdq_params* p, const void* blob_dev, int64_t M, void* Y, void* workspace,
+                      size_t ws_bytes, svdq_stream stream);
+
+/*
  * After svdq_linear: copy the quantised activations out of the workspace in
  * canonical form (synchronises `stream`).  Any output pointer may be NULL.
  *   codes   M x K host, one code per byte (INT4 int8 / NVFP4 E2M1 low nibble)
@@ -157,6 +169,10 @@ svdq_status svdq_get_status(svdq_stream stream);
 
 const char* svdq_status_string(svdq_status s);
 
+/* The CUDA error behind the most recent SVDQ_ERR_CUDA returned on this host
+ * thread ("" if none): the failing step and cudaGetErrorString's text. */
+const char* svdq_last_error_string(void);
+
 /*
  * Test hook: the GPU's own fp32 -> E2M1 and fp32 -> E4M3 conversions
  * (cvt.rn.satfinite), used to pin the host encoders.  in: n fp32 device;
@@ -164,6 +180,32 @@ const char* svdq_status_string(svdq_status s);
  */
 svdq_status svdq_probe_cvt(const float* in, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
                            svdq_stream stream);
+
+/*
+ * Test hook: the quotient v[i] / d[i] as the activation kernel computes it
+ * (one round-to-nearest reciprocal per block, then an FMA-corrected product)
+ * into q, and the IEEE round-to-nearest division into q_ieee, so that tests
+ * can check the two agree bit for bit.  All pointers: n fp32, device.
+ */
+svdq_status svdq_probe_div(const float* v, const float* d, int64_t n, float* q, float* q_ieee,
+                           svdq_stream stream);
+
+/*
+ * Measurement hook: tensor-core operation rate.  Launches `ctas` CTAs (pairs
+ * of CTAs for op 1); in each, one thread issues `iters` back-to-back tcgen05
+ * operations of kind `op` on zeroed shared memory and writes the clock64
+ * cycles it took (issue to completion) to cycles[cta] (device, ctas entries).
+ *   0 mxf4nvf4 128x256x64   1 mxf4nvf4 256x256x64 (CTA pair)
+ *   2 bf16 128x256x16       3 E4M3 128x256x32      4 s8 128x256x32
+ *   5 scale-factor copy (tcgen05.cp 32x128b.warpx4) only
+ *   6 op 0 + 12 copies (32x128b.warpx4) per 4 MMAs
+ *   7 op 0 + 6 copies (128x256b) per 4 MMAs
+ *   8 tcgen05.st 32x32b.x32 (+ wait) by 4 warps; cycles[ctas * w + cta], w = 1..4
+ *   9 op 0 while 4 other warps store 48 TMEM columns per 4 MMAs (warp cycles as op 8)
+ *   10 op 1 + 12 copies (cta_group::2 32x128b.warpx4) per 4 MMAs (CTA pair)
+ * cycles must hold 5 * ctas entries.  Time the launch with events on `stream` to get the chip-wide rate.
+ */
+svdq_status svdq_probe_tc(int op, int iters, int ctas, unsigned long long* cycles, svdq_stream stream);
 
 #ifdef __cplusplus
 }

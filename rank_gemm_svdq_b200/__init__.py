@@ -35,7 +35,10 @@ class svdq_params(ctypes.Structure):
 class SVDQError(RuntimeError):
     def __init__(self, status: int, what: str = ""):
         self.status = status
-        super().__init__(f"{what}: {status_string(status)} ({status})" if what else status_string(status))
+        msg = f"{what}: {status_string(status)} ({status})" if what else status_string(status)
+        if status == ERR_CUDA:
+            msg += f" [{_lib.svdq_last_error_string().decode()}]"
+        super().__init__(msg)
 
 
 def _load():
@@ -51,10 +54,15 @@ def _load():
         "svdq_blob_export": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
         "svdq_workspace_bytes": (sz, [P, i64]),
         "svdq_linear": (ctypes.c_int, [P, vp, vp, i64, vp, vp, sz, vp]),
+        "svdq_quantize_act": (ctypes.c_int, [P, vp, vp, i64, vp, sz, vp]),
+        "svdq_gemm": (ctypes.c_int, [P, vp, i64, vp, vp, sz, vp]),
         "svdq_export_act": (ctypes.c_int, [P, vp, i64, vp, vp, vp, vp]),
         "svdq_get_status": (ctypes.c_int, [vp]),
         "svdq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "svdq_last_error_string": (ctypes.c_char_p, []),
         "svdq_probe_cvt": (ctypes.c_int, [vp, i64, vp, vp, vp]),
+        "svdq_probe_div": (ctypes.c_int, [vp, vp, i64, vp, vp, vp]),
+        "svdq_probe_tc": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -64,8 +72,8 @@ def _load():
 
 _lib = _load()
 EXPORTED = ("svdq_blob_bytes", "svdq_prepare", "svdq_blob_check", "svdq_blob_export",
-            "svdq_workspace_bytes", "svdq_linear", "svdq_export_act", "svdq_get_status",
-            "svdq_status_string", "svdq_probe_cvt")
+            "svdq_workspace_bytes", "svdq_linear", "svdq_quantize_act", "svdq_gemm", "svdq_export_act", "svdq_get_status",
+            "svdq_status_string", "svdq_last_error_string", "svdq_probe_cvt", "svdq_probe_div", "svdq_probe_tc")
 
 
 def lib():
@@ -160,6 +168,19 @@ def linear(p: svdq_params, blob_dev, X, M: int, Y, workspace, stream=None):
     _check(st, "svdq_linear")
 
 
+def quantize_act(p: svdq_params, blob_dev, X, M: int, workspace, stream=None):
+    """Kernel 1 only: X -> quantised activations + down projection in `workspace`."""
+    _check(_lib.svdq_quantize_act(ctypes.byref(p), _ptr(blob_dev), _ptr(X), M, _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)),
+           "svdq_quantize_act")
+
+
+def gemm(p: svdq_params, blob_dev, M: int, Y, workspace, stream=None):
+    """Kernel 2 only: workspace -> Y (after quantize_act on the same stream)."""
+    _check(_lib.svdq_gemm(ctypes.byref(p), _ptr(blob_dev), M, _ptr(Y), _ptr(workspace),
+                          workspace.numel() * workspace.element_size(), _stream(stream)), "svdq_gemm")
+
+
 def export_act(p: svdq_params, workspace, M: int, stream=None):
     """Quantised activations after svdq_linear: (codes M x K, scales, u' M x r)."""
     K, r = p.K, p.rank
@@ -179,6 +200,15 @@ def get_status(stream=None) -> int:
 
 def probe_cvt(x, e2m1, e4m3, stream=None):
     _check(_lib.svdq_probe_cvt(_ptr(x), x.numel(), _ptr(e2m1), _ptr(e4m3), _stream(stream)), "svdq_probe_cvt")
+
+
+def probe_div(v, d, q, q_ieee, stream=None):
+    _check(_lib.svdq_probe_div(_ptr(v), _ptr(d), v.numel(), _ptr(q), _ptr(q_ieee), _stream(stream)),
+           "svdq_probe_div")
+
+
+def probe_tc(op: int, iters: int, ctas: int, cycles, stream=None):
+    _check(_lib.svdq_probe_tc(op, iters, ctas, _ptr(cycles), _stream(stream)), "svdq_probe_tc")
 
 
 def _stream(s):

@@ -5,19 +5,32 @@
 //   inv_lambda  K fp32                                  smoothing, device multiplies X by it
 //   l1t         r x K act_dtype (L1 transposed)          B operand of the down projection
 //   l2x         N x lrw bf16, K-major                    B operand of the up projection
+//               (NVFP4: as low-rank tiles, below; INT4: row-major)
 //               (lrw = nseg*r rounded up to 64, zero padded):
 //               bf16 X: [L2 ; L2]             (pairs with [u_hi | u_lo])
 //               fp16 X: [L2h ; L2h ; L2l]     (pairs with [u_hi | u_lo | u_hi]; L2 = L2h + L2l exactly)
-//   wq          NVFP4: N x K/2 bytes, E2M1 packed, element k in the low nibble when k is even
+//   wq          NVFP4: weight tiles (below), [N/128][K/256] x 20480 bytes
 //               INT4:  N x K bytes, the code as an E4M3 byte (exact for -8..7)
-//   ws          NVFP4: E4M3 block scales in the tcgen05 scale-factor atom layout (below)
+//   ws          NVFP4: empty (the scales live in the weight tiles)
 //               INT4:  fp32 [K/64][N]
 //   bias        N fp32
 //
 // Workspace for M tokens:
-//   xq   NVFP4: M x K/2 bytes packed E2M1;   INT4: M x K bytes (code as E4M3 byte)
-//   xs   NVFP4: scale-factor atoms for ceil(M/128)*128 rows;  INT4: fp32 [K/64][Mp], Mp = ceil(M/128)*128
+//   xq   NVFP4: activation tiles (below), [Mp/128][K/256] x 18432 bytes
+//        INT4:  M x K bytes (code as E4M3 byte)
+//   xs   NVFP4: empty;  INT4: fp32 [K/64][Mp], Mp = ceil(M/128)*128
 //   ux   M x lrw bf16: [u'_hi | u'_lo (| u'_hi) | 0 pad], u' = u / (s_gX s_gW) (NVFP4) or u (INT4)
+//        (NVFP4: as low-rank tiles over Mp rows; INT4: row-major)
+//
+// NVFP4 operand tiles (what one bulk copy brings into shared memory, ready
+// for the tensor core): 128 rows x one K slab of 256 elements.  The E2M1
+// codes (two per byte, even element in the low nibble) sit as 128 rows of
+// 128 bytes with the 128-byte swizzle -- 16-byte chunk c of row r stored at
+// chunk c ^ (r % 8) -- followed by the slab's E4M3 scale atoms:
+//   activation tile: 16384 bytes of codes + 2048 bytes of scales (its 128 rows)
+//   weight tile:     16384 bytes of codes + 4096 bytes of scales of the 256 rows
+//                    (two row blocks 2p, 2p+1) that one CTA pair multiplies
+// Low-rank tiles: 128 rows x 64 bf16 (128 bytes), same swizzle, 16384 bytes.
 //
 // Scale-factor atom layout (the operand format of tcgen05 block-scaled MMA
 // scale factors once copied to tensor memory by tcgen05.cp 32x128b.warpx4):
@@ -39,6 +52,10 @@ constexpr uint32_t kVersion = 1;
 constexpr size_t kAlign = 1024;
 constexpr int kGroupInt4 = 64;
 constexpr int kBlockFp4 = 16;
+constexpr int kTileCodes = 16384;   // 128 rows x 128 bytes
+constexpr int kATile = 18432;       // activation tile: codes + 128 rows of scales
+constexpr int kWTile = 20480;       // weight tile: codes + 256 rows of scales
+constexpr int kLRTile = 16384;      // low-rank tile: 128 rows x 64 bf16
 
 struct BlobHeader {
   uint32_t magic0, magic1, version, header_bytes;
@@ -77,9 +94,9 @@ inline BlobLayout blob_layout(const svdq_params& p) {
   L.off_l1t = off;        off = align_up(off + r * K * 2);
   L.off_l2x = off;        off = align_up(off + N * (size_t)lr_width(p) * 2);
   L.off_wq = off;
-  off = align_up(off + (p.fmt == SVDQ_NVFP4 ? N * K / 2 : N * K));
+  off = align_up(off + (p.fmt == SVDQ_NVFP4 ? (N / 128) * (K / 256) * (size_t)kWTile : N * K));
   L.off_ws = off;
-  off = align_up(off + (p.fmt == SVDQ_NVFP4 ? N * (K / kBlockFp4) : (K / kGroupInt4) * N * 4));
+  off = align_up(off + (p.fmt == SVDQ_NVFP4 ? 0 : (K / kGroupInt4) * N * 4));
   L.off_bias = off;       off = align_up(off + N * 4);
   L.total = off;
   return L;
@@ -87,21 +104,23 @@ inline BlobLayout blob_layout(const svdq_params& p) {
 
 struct WsLayout {
   size_t off_xq, off_xs, off_ux, total;
-  int64_t Mp;  // M rounded up to 128
+  int64_t Mp;  // M rounded up to the GEMM's row tile (256 NVFP4, 128 INT4)
 };
 
 inline WsLayout ws_layout(const svdq_params& p, int64_t M) {
   WsLayout L{};
   const size_t K = (size_t)p.K;
-  L.Mp = (M + 127) / 128 * 128;
+  // NVFP4 pads tokens to whole 256-row tiles (one CTA pair), INT4 to 128
+  const int64_t pad = p.fmt == SVDQ_NVFP4 ? 256 : 128;
+  L.Mp = (M + pad - 1) / pad * pad;
   const size_t Mp = (size_t)L.Mp;
   size_t off = 0;
   L.off_xq = off;
-  off = align_up(off + (p.fmt == SVDQ_NVFP4 ? (size_t)M * K / 2 : (size_t)M * K));
+  off = align_up(off + (p.fmt == SVDQ_NVFP4 ? (Mp / 128) * (K / 256) * (size_t)kATile : (size_t)M * K));
   L.off_xs = off;
-  off = align_up(off + (p.fmt == SVDQ_NVFP4 ? Mp * (K / kBlockFp4) : (K / kGroupInt4) * Mp * 4));
+  off = align_up(off + (p.fmt == SVDQ_NVFP4 ? 0 : (K / kGroupInt4) * Mp * 4));
   L.off_ux = off;
-  off = align_up(off + (size_t)M * (size_t)lr_width(p) * 2);
+  off = align_up(off + (p.fmt == SVDQ_NVFP4 ? Mp : (size_t)M) * (size_t)lr_width(p) * 2);
   L.total = off > 0 ? off : kAlign;
   return L;
 }
@@ -112,6 +131,17 @@ SVDQ_HD inline size_t sf_offset(int64_t row, int64_t blk, int64_t kblocks) {
   const int64_t atom = (row / 128) * (kblocks / 4) + blk / 4;
   const int64_t r = row % 128;
   return (size_t)(atom * 512 + (r % 32) * 16 + (r / 32) * 4 + (blk % 4));
+}
+
+// Byte offset of (row r, byte c) inside a 128 x 128-byte tile with the 128-byte swizzle.
+SVDQ_HD inline uint32_t sw128(uint32_t r, uint32_t c) {
+  return r * 128u + ((((c >> 4) ^ (r & 7u)) & 7u) << 4) + (c & 15u);
+}
+
+// Byte offset of the scale of tile row rr (0..127) and scale block j (0..15
+// inside the slab) within a tile's scale atoms.
+SVDQ_HD inline uint32_t tile_sf(uint32_t rr, uint32_t j) {
+  return (j >> 2) * 512u + (rr & 31u) * 16u + (rr >> 5) * 4u + (j & 3u);
 }
 
 }  // namespace svdq

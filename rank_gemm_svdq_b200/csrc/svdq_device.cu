@@ -20,8 +20,11 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 #include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <vector>
 
@@ -84,9 +87,31 @@ struct ActArgs {
   uint16_t* ux;
 };
 
-constexpr int kActRows = 32;     // tokens per CTA
+constexpr int kActRows = 16;     // tokens per CTA
 constexpr int kActChunk = 256;   // K elements per step
 constexpr int kActStride = kActChunk + 8;  // padded smem row (bf16/fp16 elements)
+
+// Correctly rounded fp32 quotient v / d given r = RN(1 / d): q = RN(v r) is
+// within one ulp, the remainder e = v - q d is exact with one FMA, and
+// RN(q + e r) is the correctly rounded quotient (Markstein's theorem; see
+// Muller et al., Handbook of Floating-Point Arithmetic, the FMA-based division
+// section).  Valid while the remainder is representable and nothing
+// overflows: the callers use it only for 2^-100 <= d <= 2^125 (recip_ok), and
+// for quotients below 2^-2 (where the exact remainder may underflow) every
+// 4-bit code is zero either way, with the sign preserved.
+__device__ __forceinline__ bool recip_ok(float d) { return d >= 0x1p-100f && d <= 0x1p+125f; }
+
+__device__ __forceinline__ float div_by_recip(float v, float d, float r) {
+  const float q = __fmul_rn(v, r);
+  const float e = __fmaf_rn(-q, d, v);
+  return __fmaf_rn(e, r, q);
+}
+
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& a0, uint32_t& a1, uint32_t& a2,
                                             uint32_t& a3) {
@@ -117,112 +142,169 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a
   }
 }
 
-// One CTA = 32 tokens x all of K, 8 warps.  Warp w owns tokens 4w..4w+3; lane
-// l owns elements 8l..8l+7 of each 256-wide chunk (one 16-byte load per row).
+template <int DT>
+__device__ __forceinline__ uint32_t pack_half2_rn(float lo, float hi) {
+  if constexpr (DT == SVDQ_BF16) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  } else {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+}
+
+// Quantise 16 consecutive smoothed activations of one token (one NVFP4
+// block, or a quarter of an INT4 group of 64 spread over 4 lanes) and store
+// codes / scales.
+template <int FMT>
+__device__ __forceinline__ void quantize16(const float (&xh)[16], int64_t m, int kk, const ActArgs& a,
+                                           float s_gx, float six_sg, float r6) {
+  const int K = a.K;
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(xh[i]));
+  if constexpr (FMT == SVDQ_NVFP4) {
+    const float ratio = r6 != 0.0f ? div_by_recip(amax, six_sg, r6) : __fdiv_rn(amax, six_sg);
+    const uint32_t e = cvt_e4m3x2(0.0f, ratio) & 0xFFu;
+    const float d = __fmul_rn(e4m3_val(e), s_gx);
+    uint32_t p0 = 0, p1 = 0;
+    if (d != 0.0f) {
+      if (recip_ok(d)) {
+        const float rd = __frcp_rn(d);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          p0 |= cvt_e2m1x2(div_by_recip(xh[2 * i + 1], d, rd), div_by_recip(xh[2 * i], d, rd)) << (8 * i);
+          p1 |= cvt_e2m1x2(div_by_recip(xh[2 * i + 9], d, rd), div_by_recip(xh[2 * i + 8], d, rd)) << (8 * i);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          p0 |= cvt_e2m1x2(__fdiv_rn(xh[2 * i + 1], d), __fdiv_rn(xh[2 * i], d)) << (8 * i);
+          p1 |= cvt_e2m1x2(__fdiv_rn(xh[2 * i + 9], d), __fdiv_rn(xh[2 * i + 8], d)) << (8 * i);
+        }
+      }
+    }
+    // activation tile (m / 128, slab): swizzled codes, then the slab's scale atoms
+    if (m < a.Mp) {
+      uint8_t* tile = a.xq + ((size_t)(m >> 7) * (K / 256) + kk / 256) * kATile;
+      const uint32_t rr = (uint32_t)(m & 127);
+      *reinterpret_cast<uint2*>(tile + sw128(rr, (uint32_t)(kk & 255) >> 1)) = make_uint2(p0, p1);
+      tile[kTileCodes + tile_sf(rr, (uint32_t)(kk & 255) >> 4)] = (uint8_t)e;
+    }
+  } else {
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // group of 64 = 4 lanes
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    const float s = __fdiv_rn(amax, 7.0f);
+    uint32_t w[8];
+    if (amax == 0.0f) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = 0;
+    } else {
+      const bool fast = recip_ok(s);
+      const float rs = fast ? __frcp_rn(s) : 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float t0 = fast ? div_by_recip(xh[2 * i], s, rs) : __fdiv_rn(xh[2 * i], s);
+        const float t1 = fast ? div_by_recip(xh[2 * i + 1], s, rs) : __fdiv_rn(xh[2 * i + 1], s);
+        const int q0 = min(7, max(-8, __float2int_rn(t0)));
+        const int q1 = min(7, max(-8, __float2int_rn(t1)));
+        w[i] = cvt_e4m3x2((float)q1, (float)q0);
+      }
+    }
+    if (m < a.M)
+      *reinterpret_cast<uint4*>(a.xq + (size_t)m * K + kk) =
+          make_uint4(w[0] | (w[1] << 16), w[2] | (w[3] << 16), w[4] | (w[5] << 16), w[6] | (w[7] << 16));
+    if (((threadIdx.x & 3) == 0) && m < a.Mp) reinterpret_cast<float*>(a.xs)[(size_t)(kk / 64) * a.Mp + m] = s;
+  }
+}
+
+// One CTA = 16 tokens x all of K, 8 warps.  Per 256-wide chunk, warp w owns
+// tokens 2w (lanes 0-15) and 2w+1 (lanes 16-31); lane l owns elements
+// 16(l%16) .. 16(l%16)+15 (two 16-byte loads).  The next chunk's loads are
+// issued before the current chunk is processed; the X^16 and L1 tiles in
+// shared memory are double-buffered so a chunk costs one __syncthreads.  The
+// down projection u = X^16 L1 runs on mma.sync (m16n8k16, fp32 accumulate),
+// one n8 tile of u per warp.
 template <int FMT, int DT>
 __global__ void __launch_bounds__(256) act_quant_kernel(const ActArgs a) {
   extern __shared__ __align__(16) uint16_t act_smem[];
-  uint16_t* xs16 = act_smem;                          // [32][kActStride]
-  uint16_t* l1s = act_smem + kActRows * kActStride;   // [r][kActStride]
+  const int K = a.K, r = a.r;
+  uint16_t* const xs16_base = act_smem;
+  uint16_t* const l1s_base = act_smem + 2 * kActRows * kActStride;
+  auto xs16 = [&](int b) { return xs16_base + b * kActRows * kActStride; };
+  auto l1sb = [&](int b) { return l1s_base + b * r * kActStride; };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t m0 = (int64_t)blockIdx.x * kActRows;
-  const int K = a.K, r = a.r;
   const float s_gx = a.hdr->s_gx;
   const float six_sg = __fmul_rn(6.0f, s_gx);
+  const float r6 = recip_ok(six_sg) ? __frcp_rn(six_sg) : 0.0f;
   const float inv_alpha = FMT == SVDQ_NVFP4 ? 1.0f / (a.hdr->s_gx * a.hdr->s_gw) : 1.0f;
+  const int n_tiles = r / 8;   // one m16 tile (16 tokens) x r/8 n8 tiles
 
-  // u tiles: (32/16) x (r/8) tiles of m16n8, spread over the 8 warps
-  const int n_tiles = 2 * (r / 8);
-  float acc[4][4];
+  float acc[2][4];
 #pragma unroll
-  for (int t = 0; t < 4; ++t)
+  for (int t = 0; t < 2; ++t)
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[t][i] = 0.0f;
 
-  for (int k0 = 0; k0 < K; k0 += kActChunk) {
-    // stage this chunk of L1^T (r rows x 256) in shared memory
+  const int rw = warp * 2 + (lane >> 4);     // token row inside the CTA
+  const int64_t m = m0 + rw;
+  const int col = (lane & 15) * 16;          // element offset inside the chunk
+  const bool live = m < a.M;
+  const uint16_t* xrow = a.X + (live ? m : 0) * K + col;
+  uint4 xc[2], xn[2];
+  xc[0] = live ? __ldg(reinterpret_cast<const uint4*>(xrow)) : make_uint4(0, 0, 0, 0);
+  xc[1] = live ? __ldg(reinterpret_cast<const uint4*>(xrow + 8)) : make_uint4(0, 0, 0, 0);
+
+  // L1^T chunks arrive by cp.async one chunk ahead (issued right after the
+  // chunk barrier, when the other buffer is no longer read)
+  auto stage_l1 = [&](int chunk, int b) {
     for (int idx = tid; idx < r * (kActChunk / 8); idx += 256) {
       const int i = idx / (kActChunk / 8), c8 = idx % (kActChunk / 8);
-      *reinterpret_cast<uint4*>(l1s + i * kActStride + c8 * 8) =
-          __ldg(reinterpret_cast<const uint4*>(a.l1t + (size_t)i * K + k0 + c8 * 8));
+      cp_async_16(l1sb(b) + i * kActStride + c8 * 8, a.l1t + (size_t)i * K + chunk * kActChunk + c8 * 8);
     }
-    const int kk = k0 + lane * 8;
-    const float4 il0 = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + kk));
-    const float4 il1 = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + kk + 4));
-    const float il[8] = {il0.x, il0.y, il0.z, il0.w, il1.x, il1.y, il1.z, il1.w};
+    cp_async_commit();
+  };
+  stage_l1(0, 0);
 
-    uint4 xin[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t m = m0 + warp * 4 + j;
-      xin[j] = m < a.M ? __ldg(reinterpret_cast<const uint4*>(a.X + m * K + kk)) : make_uint4(0, 0, 0, 0);
+  const int nchunks = K / kActChunk;
+  for (int c = 0; c < nchunks; ++c) {
+    const int k0 = c * kActChunk;
+    const int buf = c & 1;
+    if (c + 1 < nchunks) {
+      xn[0] = live ? __ldg(reinterpret_cast<const uint4*>(xrow + k0 + kActChunk)) : make_uint4(0, 0, 0, 0);
+      xn[1] = live ? __ldg(reinterpret_cast<const uint4*>(xrow + k0 + kActChunk + 8)) : make_uint4(0, 0, 0, 0);
     }
+    const int kk = k0 + col;
+    float il[16];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int rw = warp * 4 + j;
-      const int64_t m = m0 + rw;
-      const uint16_t* xh16 = reinterpret_cast<const uint16_t*>(&xin[j]);
-      float xh[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) xh[i] = __fmul_rn(half_to_f32<DT>(xh16[i]), il[i]);
-
-      float amax = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(xh[i]));
-
-      if constexpr (FMT == SVDQ_NVFP4) {
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));       // block of 16 = 2 lanes
-        const float ratio = __fdiv_rn(amax, six_sg);
-        const uint32_t e = cvt_e4m3x2(0.0f, ratio) & 0xFFu;
-        const float d = __fmul_rn(e4m3_val(e), s_gx);
-        uint32_t packed = 0;
-        if (d != 0.0f) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            packed |= cvt_e2m1x2(__fdiv_rn(xh[2 * i + 1], d), __fdiv_rn(xh[2 * i], d)) << (8 * i);
-        }
-        if (m < a.M) *reinterpret_cast<uint32_t*>(a.xq + (size_t)m * (K / 2) + kk / 2) = packed;
-        if ((lane & 1) == 0 && m < a.Mp) a.xs[sf_offset(m, kk / 16, K / 16)] = (uint8_t)e;
-      } else {
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));       // group of 64 = 8 lanes
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-        const float s = __fdiv_rn(amax, 7.0f);
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          int q0 = 0, q1 = 0;
-          if (amax != 0.0f) {
-            q0 = min(7, max(-8, __float2int_rn(__fdiv_rn(xh[2 * i], s))));
-            q1 = min(7, max(-8, __float2int_rn(__fdiv_rn(xh[2 * i + 1], s))));
-          }
-          w[i] = cvt_e4m3x2((float)q1, (float)q0);
-        }
-        if (m < a.M)
-          *reinterpret_cast<uint2*>(a.xq + (size_t)m * K + kk) =
-              make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
-        if ((lane & 7) == 0 && m < a.Mp)
-          reinterpret_cast<float*>(a.xs)[(size_t)(kk / 64) * a.Mp + m] = s;
-      }
-      // X^ rounded to the 16-bit dtype: the low-rank branch's input
-      uint4 o;
-      uint16_t* o16 = reinterpret_cast<uint16_t*>(&o);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) o16[i] = f32_to_half_rn<DT>(xh[i]);
-      *reinterpret_cast<uint4*>(xs16 + rw * kActStride + lane * 8) = o;
+    for (int i = 0; i < 4; ++i) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + kk + 4 * i));
+      il[4 * i] = f.x; il[4 * i + 1] = f.y; il[4 * i + 2] = f.z; il[4 * i + 3] = f.w;
     }
+    const uint16_t* x16 = reinterpret_cast<const uint16_t*>(xc);
+    float xh[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) xh[i] = __fmul_rn(half_to_f32<DT>(x16[i]), il[i]);
+    quantize16<FMT>(xh, m, kk, a, s_gx, six_sg, r6);
+    uint4 o0, o1;
+    o0.x = pack_half2_rn<DT>(xh[0], xh[1]);   o0.y = pack_half2_rn<DT>(xh[2], xh[3]);
+    o0.z = pack_half2_rn<DT>(xh[4], xh[5]);   o0.w = pack_half2_rn<DT>(xh[6], xh[7]);
+    o1.x = pack_half2_rn<DT>(xh[8], xh[9]);   o1.y = pack_half2_rn<DT>(xh[10], xh[11]);
+    o1.z = pack_half2_rn<DT>(xh[12], xh[13]); o1.w = pack_half2_rn<DT>(xh[14], xh[15]);
+    uint4* dst = reinterpret_cast<uint4*>(xs16(buf) + rw * kActStride + col);
+    dst[0] = o0;
+    dst[1] = o1;
+    cp_async_wait_all();
     __syncthreads();
-
-    // u += X^16[32 x 256] * L1[256 x r]   (mma.sync m16n8k16, fp32 accumulate)
+    if (c + 1 < nchunks) stage_l1(c + 1, buf ^ 1);
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const int tile = warp + 8 * t;
-      if (tile < n_tiles) {
-        const int mt = tile & 1, nt = tile >> 1;
-        const uint32_t a_base =
-            smem_u32(xs16 + (mt * 16 + (lane & 15)) * kActStride + (lane >> 4) * 8);
-        const uint32_t b_base = smem_u32(l1s + (nt * 8 + (lane & 7)) * kActStride + ((lane >> 3) & 1) * 8);
+    for (int t = 0; t < 2; ++t) {
+      const int nt = warp + 8 * t;
+      if (nt < n_tiles) {
+        const uint32_t a_base = smem_u32(xs16(buf) + (lane & 15) * kActStride + (lane >> 4) * 8);
+        const uint32_t b_base = smem_u32(l1sb(buf) + (nt * 8 + (lane & 7)) * kActStride + ((lane >> 3) & 1) * 8);
 #pragma unroll 4
         for (int ks = 0; ks < kActChunk / 16; ++ks) {
           uint32_t a0, a1, a2, a3, b0, b1;
@@ -232,31 +314,40 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const ActArgs a) {
         }
       }
     }
-    __syncthreads();
+    xc[0] = xn[0];
+    xc[1] = xn[1];
   }
 
-  // u' = u * inv_alpha, split into bf16 hi + lo: [hi | lo (| hi) | 0 pad]
+  // u' = u * inv_alpha, split into bf16 hi + lo: [hi | lo (| hi) | 0 pad];
+  // NVFP4 keeps it as swizzled low-rank tiles over the padded rows
+  const int64_t u_rows = FMT == SVDQ_NVFP4 ? a.Mp : a.M;
+  auto ux_at = [&](int64_t mm, int e) -> uint32_t* {
+    if constexpr (FMT == SVDQ_NVFP4) {
+      uint8_t* tile = reinterpret_cast<uint8_t*>(a.ux) + ((size_t)(mm >> 7) * (a.lrw / 64) + e / 64) * kLRTile;
+      return reinterpret_cast<uint32_t*>(tile + sw128((uint32_t)(mm & 127), (uint32_t)(e & 63) * 2));
+    } else {
+      return reinterpret_cast<uint32_t*>(a.ux + (size_t)mm * a.lrw + e);
+    }
+  };
 #pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    const int tile = warp + 8 * t;
-    if (tile < n_tiles) {
-      const int mt = tile & 1, nt = tile >> 1;
-      const int col = nt * 8 + 2 * (lane & 3);
+  for (int t = 0; t < 2; ++t) {
+    const int nt = warp + 8 * t;
+    if (nt < n_tiles) {
+      const int ucol = nt * 8 + 2 * (lane & 3);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        const int64_t m = m0 + mt * 16 + (lane >> 2) + half * 8;
-        if (m < a.M) {
+        const int64_t mu = m0 + (lane >> 2) + half * 8;
+        if (mu < u_rows) {
           uint16_t hi[2], lo[2];
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const float v = acc[t][half * 2 + c] * inv_alpha;
-            hi[c] = bf16_rn(v);
-            lo[c] = bf16_rn(v - __uint_as_float((uint32_t)hi[c] << 16));
+          for (int cc = 0; cc < 2; ++cc) {
+            const float v = acc[t][half * 2 + cc] * inv_alpha;
+            hi[cc] = bf16_rn(v);
+            lo[cc] = bf16_rn(v - __uint_as_float((uint32_t)hi[cc] << 16));
           }
-          uint16_t* row = a.ux + (size_t)m * a.lrw;
-          *reinterpret_cast<uint32_t*>(row + col) = hi[0] | ((uint32_t)hi[1] << 16);
-          *reinterpret_cast<uint32_t*>(row + r + col) = lo[0] | ((uint32_t)lo[1] << 16);
-          if (a.nseg == 3) *reinterpret_cast<uint32_t*>(row + 2 * r + col) = hi[0] | ((uint32_t)hi[1] << 16);
+          *ux_at(mu, ucol) = hi[0] | ((uint32_t)hi[1] << 16);
+          *ux_at(mu, r + ucol) = lo[0] | ((uint32_t)lo[1] << 16);
+          if (a.nseg == 3) *ux_at(mu, 2 * r + ucol) = hi[0] | ((uint32_t)hi[1] << 16);
         }
       }
     }
@@ -264,9 +355,9 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const ActArgs a) {
   const int used = a.nseg * r;
   const int pad = a.lrw - used;
   if (pad > 0) {
-    for (int idx = tid; idx < kActRows * pad; idx += 256) {
-      const int64_t m = m0 + idx / pad;
-      if (m < a.M) a.ux[(size_t)m * a.lrw + used + idx % pad] = 0;
+    for (int idx = tid; idx < kActRows * (pad / 2); idx += 256) {
+      const int64_t mu = m0 + idx / (pad / 2);
+      if (mu < u_rows) *ux_at(mu, used + 2 * (idx % (pad / 2))) = 0;
     }
   }
 }
@@ -316,149 +407,245 @@ __device__ __forceinline__ void store_row32(uint16_t* dst, const float* v, const
   for (int j = 0; j < 4; ++j) d4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
 }
 
-// ------------------------------------------------------------ kernel 2, NVFP4
-// One CTA per 128 x 256 output tile.  Warp 0: TMA producer.  Warp 1: TMEM
-// owner and MMA issuer.  Warps 2-5: epilogue (TMEM lane quarter = warp % 4).
-// TMEM: columns [0,256) accumulator; [256,288) and [288,352) two buffers of
-// activation / weight scale factors.
-constexpr int kSfaBytes = 4 * 512;                 // 128 rows x 16 scale blocks
-constexpr int kSfbBytes = 2 * 4 * 512;             // 256 rows x 16 scale blocks
-constexpr int kFp4StageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;   // 55296
+// ------------------------------------------------------------ kernel 2, NVFP4 (CTA pairs)
+// Persistent, clusters of 2 CTAs; each pair walks 256 x 256 output tiles
+// (pair p: tile p, p + pairs, ..., n fastest).  In a pair, CTA r holds A rows
+// [128r, 128r + 128) of the tile and B rows (output features) [128r, 128r+128)
+// in its shared memory; the leader (rank 0) issues cta_group::2 MMAs
+// (M = 256, N = 256) that read both CTAs' operands and accumulate each CTA's
+// 128 rows in its own TMEM, so every B byte is fetched once per pair.
+//
+// Data path: the operands are stored as ready-made tiles (swizzled codes
+// followed by their scale atoms), so a K slab of one CTA is two bulk copies
+// (activation tile 18 KB, weight tile 20 KB) into a 5-deep stage ring.  Each
+// CTA's copies signal its own `landed` barrier.
+// Scale factors: four scale warps per CTA (one per TMEM lane quarter) wait
+// for their stage to land, copy its scale atoms to that stage's TMEM slot
+// with tcgen05.st, and arrive on the leader's `ready` barrier; the MMA
+// issuer waits only for `ready` (all eight scale warps of both CTAs), which
+// implies both CTAs' bytes landed.  The leader's tcgen05.commit (CTA mask
+// 0b11) frees the stage in both CTAs.  A stage refills only after its MMAs
+// completed, so the TMEM scale slot needs no separate release.
+//
+// Warps (four warpgroups, register budgets set with setmaxnreg so that the
+// sum fits the 64K-register file): 0 producer, 1 TMEM owner + MMA issuer
+// (leader), 2-3 idle [56 regs]; 4-7 scale warps [80]; 8-15 epilogue, lane
+// quarter warp % 4, column half (warp - 8) / 4 [184].  The
+// epilogue copies its 128 accumulator columns to registers with four
+// back-to-back tcgen05.ld, releases TMEM, then adds alpha / bias and stores
+// bf16 rows while the next tile runs.
+// TMEM: [0,256) accumulator; stage s scale slot at 256 + 48 s (SFA 16, SFB 32 columns).
+constexpr int kS_SFA = kTileCodes;                 // stage: [A codes | SFA | B codes | SFB]
+constexpr int kS_B = kATile;
+constexpr int kS_SFB = kATile + kTileCodes;
+constexpr int kS_Size = kATile + kWTile;           // 38912
+constexpr int kP_Stages = 5;
+constexpr int kEpiWarps = 8;
+constexpr int kP_Threads = 16 * 32;
+constexpr int kP_Smem = kP_Stages * kS_Size + kEpiWarps * 128 * 4 + 1024;
 
-__global__ void __launch_bounds__(192, 1)
-    gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                      const __grid_constant__ CUtensorMap tm_ua, const __grid_constant__ CUtensorMap tm_ub,
-                      const GemmArgs g) {
+struct PairArgs {
+  int64_t M, Mp;
+  int N, K;
+  int lr_iters;            // low-rank K steps (64 bf16 each)
+  int k_iters;             // 4-bit K slabs (256 elements each)
+  const uint8_t* atiles;   // activation tiles [Mp/128][K/256]
+  const uint8_t* wtiles;   // weight tiles [N/128][K/256]
+  const uint8_t* utiles;   // low-rank input tiles [Mp/128][lr_iters]
+  const uint8_t* l2tiles;  // low-rank weight tiles [N/128][lr_iters]
+  const float* bias;
+  const BlobHeader* hdr;
+  uint16_t* Y;
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
+    gemm_nvfp4_pair_kernel(const PairArgs g) {
   extern __shared__ __align__(1024) uint8_t gsmem_raw[];
-  __shared__ uint64_t full_bar[kStages], empty_bar[kStages], accum_bar;
+  __shared__ uint64_t landed_bar[kP_Stages], empty_bar[kP_Stages], ready_bar[kP_Stages], accf_bar, acce_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
+  float* bias_smem = reinterpret_cast<float*>(smem + kP_Stages * kS_Size);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nt = blockIdx.x, mt = blockIdx.y;
-  const int n0 = nt * kBN;
-  const int64_t m0 = (int64_t)mt * kBM;
-  const int total = g.lr_iters + g.k_iters;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, pairs = gridDim.x >> 1;
+  const int n_tiles = g.N / 256;
+  const int num_tiles = n_tiles * (int)(g.Mp / 256);
+  const int per_tile = g.lr_iters + g.k_iters;
+  const int ksl = g.K / 256;
   volatile int* abort_flag = &abort_sh;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
-    mbar_init(&accum_bar, 1);
+    for (int s = 0; s < kP_Stages; ++s) {
+      mbar_init(&landed_bar[s], 1); mbar_init(&empty_bar[s], 1); mbar_init(&ready_bar[s], 2 * 4);
+    }
+    mbar_init(&accf_bar, 1);
+    mbar_init(&acce_bar, 2 * kEpiWarps);
     abort_sh = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tm_a); prefetch_tmap(&tm_b);
-    if (g.lr_iters) { prefetch_tmap(&tm_ua); prefetch_tmap(&tm_ub); }
-  }
-  if (warp == 1) { tmem_alloc(&tmem_base_sh, 512); tmem_relinquish(); }
+  if (warp == 1) { tmem_alloc_pair(&tmem_base_sh, 512); tmem_relinquish_pair(); }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
   const uint32_t tbase = tmem_base_sh;
+  const uint32_t peer_abort = mapa_shared(smem_u32(&abort_sh), rank ^ 1u);
+  auto give_up_both = [&]() { st_cluster_u32(peer_abort, 1u); };
 
   if (warp == 0) {
+    regs_dec<56>();
     if (lane == 0) {
-      int issued = 0;
-      for (int it = 0; it < total; ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        if (!mbar_wait(&empty_bar[s], ph ^ 1, abort_flag)) break;
-        uint8_t* st = smem + s * kFp4StageBytes;
-        if (it < g.lr_iters) {
-          mbar_arrive_expect_tx(&full_bar[s], kABytes + kBBytes);
-          tma_load_2d(st, &tm_ua, &full_bar[s], it * 64, (int)m0);
-          tma_load_2d(st + kABytes, &tm_ub, &full_bar[s], it * 64, n0);
-        } else {
-          const int kt = it - g.lr_iters;
-          const int katoms = g.K / 64;
-          mbar_arrive_expect_tx(&full_bar[s], kFp4StageBytes);
-          tma_load_2d(st, &tm_a, &full_bar[s], kt * 128, (int)m0);
-          tma_load_2d(st + kABytes, &tm_b, &full_bar[s], kt * 128, n0);
-          uint8_t* sf = st + kABytes + kBBytes;
-          bulk_load(sf, g.sfa + ((size_t)mt * katoms + kt * 4) * 512, kSfaBytes, &full_bar[s]);
-          bulk_load(sf + kSfaBytes, g.sfb + ((size_t)(2 * nt) * katoms + kt * 4) * 512, 2048, &full_bar[s]);
-          bulk_load(sf + kSfaBytes + 2048, g.sfb + ((size_t)(2 * nt + 1) * katoms + kt * 4) * 512, 2048,
-                    &full_bar[s]);
+      int it = 0, issued = 0;
+      bool dead = false;
+      for (int tile = pair; tile < num_tiles && !dead; tile += pairs) {
+        const int mt = tile / n_tiles, nt = tile % n_tiles;
+        const size_t mb = (size_t)(2 * mt + (int)rank), nb = (size_t)(2 * nt + (int)rank);
+        for (int j = 0; j < per_tile; ++j, ++it) {
+          const int s = it % kP_Stages;
+          if (!mbar_wait(&empty_bar[s], ((it / kP_Stages) & 1) ^ 1, abort_flag)) { give_up_both(); dead = true; break; }
+          uint8_t* st = smem + s * kS_Size;
+          if (j < g.lr_iters) {
+            mbar_arrive_expect_tx(&landed_bar[s], 2 * kLRTile);
+            bulk_load(st, g.utiles + (mb * g.lr_iters + j) * kLRTile, kLRTile, &landed_bar[s]);
+            bulk_load(st + kS_B, g.l2tiles + (nb * g.lr_iters + j) * kLRTile, kLRTile, &landed_bar[s]);
+          } else {
+            const int kt = j - g.lr_iters;
+            mbar_arrive_expect_tx(&landed_bar[s], kS_Size);
+            bulk_load(st, g.atiles + (mb * ksl + kt) * kATile, kATile, &landed_bar[s]);
+            bulk_load(st + kS_B, g.wtiles + (nb * ksl + kt) * kWTile, kWTile, &landed_bar[s]);
+          }
+          issued = it + 1;
         }
-        issued = it + 1;
       }
       if (*abort_flag) {
-        // let the copies already issued land before the CTA exits
-        for (int it = issued - 1; it >= 0 && it >= issued - kStages; --it)
-          mbar_drain(&full_bar[it % kStages], (it / kStages) & 1);
+        for (int i = issued - 1; i >= 0 && i >= issued - kP_Stages; --i)
+          mbar_drain(&landed_bar[i % kP_Stages], (i / kP_Stages) & 1);
       }
     }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t id_lr = idesc_f16_bf16(kBM, kBN);
-      const uint32_t id_f4 = idesc_nvf4(kBM, kBN);
-      for (int it = 0; it < total; ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        if (!mbar_wait(&full_bar[s], ph, abort_flag)) break;
+  } else if (warp < 4) {
+    regs_dec<56>();
+    if (warp == 1 && leader && lane == 0) {
+      const uint32_t id_lr = idesc_f16_bf16(256, 256);
+      const uint32_t id_f4 = idesc_nvf4(256, 256);
+      int it = 0, tcount = 0;
+      bool dead = false;
+      for (int tile = pair; tile < num_tiles && !dead; tile += pairs, ++tcount) {
+        if (!mbar_wait(&acce_bar, (tcount & 1) ^ 1, abort_flag)) { give_up_both(); break; }
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + s * kFp4StageBytes);
-        const uint32_t b_addr = a_addr + kABytes;
-        if (it < g.lr_iters) {
+        for (int j = 0; j < per_tile; ++j, ++it) {
+          const int s = it % kP_Stages;
+          if (!mbar_wait(&ready_bar[s], (it / kP_Stages) & 1, abort_flag)) { give_up_both(); dead = true; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * kS_Size);
+          const uint32_t b_addr = a_addr + kS_B;
+          if (j < g.lr_iters) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            mma_f16(tbase, desc_k_sw128(a_addr + 32 * j), desc_k_sw128(b_addr + 32 * j), id_lr,
-                    (it | j) != 0);
-        } else {
-          const int kt = it - g.lr_iters;
-          const uint32_t sfa_t = tbase + 256 + 16 * (kt & 1);
-          const uint32_t sfb_t = tbase + 288 + 32 * (kt & 1);
-          const uint32_t sf_addr = b_addr + kBBytes;
+            for (int q = 0; q < 4; ++q)
+              mma_f16_pair(tbase, desc_k_sw128(a_addr + 32 * q), desc_k_sw128(b_addr + 32 * q), id_lr,
+                           (j | q) != 0);
+          } else {
+            const uint32_t sfa_t = tbase + 256 + 48 * s;
+            const uint32_t sfb_t = sfa_t + 16;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tmem_cp_32x128b_x4(sfa_t + 4 * j, desc_sf_32x16(sf_addr + 512 * j));
-            tmem_cp_32x128b_x4(sfb_t + 8 * j, desc_sf_32x16(sf_addr + kSfaBytes + 512 * j));
-            tmem_cp_32x128b_x4(sfb_t + 8 * j + 4, desc_sf_32x16(sf_addr + kSfaBytes + 2048 + 512 * j));
+            for (int q = 0; q < 4; ++q)
+              mma_nvf4_pair(tbase, desc_k_sw128(a_addr + 32 * q), desc_k_sw128(b_addr + 32 * q), id_f4,
+                            sfa_t + 4 * q, sfb_t + 8 * q, (j | q) != 0);
           }
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            mma_nvf4(tbase, desc_k_sw128(a_addr + 32 * j), desc_k_sw128(b_addr + 32 * j), id_f4,
-                     sfa_t + 4 * j, sfb_t + 8 * j, (it | j) != 0);
+          mma_commit_pair(&empty_bar[s], 0x3);
         }
-        mma_commit(&empty_bar[s]);
+        if (!dead) mma_commit_pair(&accf_bar, 0x3);
       }
-      mma_commit(&accum_bar);
-      if (*abort_flag) mbar_drain(&accum_bar, 0);
+      if (*abort_flag) {
+        mma_commit_pair(&accf_bar, 0x3);
+        mbar_drain(&accf_bar, tcount & 1);
+      }
+    }
+  } else if (warp < 8) {
+    regs_dec<80>();
+    // scale warps: landed stage -> this CTA's TMEM lane quarter of the stage's scale slot
+    const int q = warp & 3;
+    const uint32_t lane_base = tbase + ((uint32_t)(q * 32) << 16);
+    int it = 0;
+    bool dead = false;
+    for (int tile = pair; tile < num_tiles && !dead; tile += pairs) {
+      for (int j = 0; j < per_tile; ++j, ++it) {
+        const int s = it % kP_Stages;
+        if (!mbar_wait(&landed_bar[s], (it / kP_Stages) & 1, abort_flag)) { give_up_both(); dead = true; break; }
+        if (j >= g.lr_iters) {
+          const uint8_t* st = smem + s * kS_Size;
+          uint32_t wa[16], wb[32];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint4 x = *reinterpret_cast<const uint4*>(st + kS_SFA + 512 * k + lane * 16);
+            wa[4 * k] = x.x; wa[4 * k + 1] = x.y; wa[4 * k + 2] = x.z; wa[4 * k + 3] = x.w;
+            const uint4 y0 = *reinterpret_cast<const uint4*>(st + kS_SFB + 512 * k + lane * 16);
+            const uint4 y1 = *reinterpret_cast<const uint4*>(st + kS_SFB + 2048 + 512 * k + lane * 16);
+            wb[8 * k] = y0.x; wb[8 * k + 1] = y0.y; wb[8 * k + 2] = y0.z; wb[8 * k + 3] = y0.w;
+            wb[8 * k + 4] = y1.x; wb[8 * k + 5] = y1.y; wb[8 * k + 6] = y1.z; wb[8 * k + 7] = y1.w;
+          }
+          tc_fence_after();
+          tmem_st_16cols(lane_base + 256 + 48 * s, wa);
+          tmem_st_32cols(lane_base + 256 + 48 * s + 16, wb);
+          tmem_st_wait();
+          tc_fence_before();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&ready_bar[s]), 0));
+      }
     }
   } else {
-    // epilogue: warps 2..5
+    regs_inc<184>();
+    // epilogue warps 8..15 (both CTAs)
     const int q = warp & 3;
-    const bool ok = mbar_wait(&accum_bar, 0, abort_flag);
-    tc_fence_after();
-    if (ok) {
-      const float alpha = g.hdr->s_gx * g.hdr->s_gw;
-      const int64_t m = m0 + q * 32 + lane;
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld_32cols(tbase + ((uint32_t)(q * 32) << 16) + c * 32, v);
-        tmem_ld_wait();
-        if (m < g.M) {
-          float bias[32], f[32];
+    const int h = (warp - 8) >> 2;
+    const uint32_t taddr = tbase + ((uint32_t)(q * 32) << 16) + h * 128;
+    const uint32_t acce_leader = mapa_shared(smem_u32(&acce_bar), 0);
+    const float alpha = g.hdr->s_gx * g.hdr->s_gw;
+    float* bsm = bias_smem + (warp - 8) * 128;
+    int tcount = 0;
+    for (int tile = pair; tile < num_tiles; tile += pairs, ++tcount) {
+      const int mt = tile / n_tiles, nt = tile % n_tiles;
+      const int col0 = nt * 256 + h * 128;
+      *reinterpret_cast<float4*>(bsm + lane * 4) = __ldg(reinterpret_cast<const float4*>(g.bias + col0 + lane * 4));
+      __syncwarp();
+      if (!mbar_wait(&accf_bar, tcount & 1, abort_flag)) { give_up_both(); break; }
+      tc_fence_after();
+      uint32_t v[128];
+      tmem_ld_32cols(taddr + 0, *reinterpret_cast<uint32_t(*)[32]>(v + 0));
+      tmem_ld_32cols(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      tmem_ld_32cols(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
+      tmem_ld_32cols(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acce_leader);
+      const int64_t m = (int64_t)mt * 256 + 128 * rank + q * 32 + lane;
+      if (m < g.M) {
+        uint4* dst = reinterpret_cast<uint4*>(g.Y + (size_t)m * g.N + col0);
 #pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            const float4 b4 = __ldg(reinterpret_cast<const float4*>(g.bias + n0 + c * 32 + j));
-            bias[j] = b4.x; bias[j + 1] = b4.y; bias[j + 2] = b4.z; bias[j + 3] = b4.w;
+        for (int c = 0; c < 16; ++c) {
+          uint32_t w[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int e = c * 8 + 2 * j;
+            const float y0 = fmaf(alpha, __uint_as_float(v[e]), bsm[e]);
+            const float y1 = fmaf(alpha, __uint_as_float(v[e + 1]), bsm[e + 1]);
+            w[j] = (uint32_t)bf16_rn(y0) | ((uint32_t)bf16_rn(y1) << 16);
           }
-#pragma unroll
-          for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
-          store_row32(g.Y + (size_t)m * g.N + n0 + c * 32, f, bias, alpha);
+          dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
+      __syncwarp();
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tbase, 512);
+    tmem_dealloc_pair(tbase, 512);
   }
 }
 
@@ -693,6 +880,145 @@ __global__ void probe_cvt_kernel(const float* in, int64_t n, uint8_t* e2m1, uint
   }
 }
 
+
+// ------------------------------------------------------------ tensor-core rate probe
+// Measures the issue-limited throughput of tcgen05 operations on this GPU:
+// one thread per CTA issues `iters` operations back to back on zeroed shared
+// memory, then waits (bounded) for their completion.  Used for the roofline
+// denominators (dense FP4 / FP8 / INT8 / BF16 tensor peaks as this part runs
+// them) and to cost the scale-factor copies of the block-scaled GEMM.
+//   op 0  kind::mxf4nvf4 block16, M=128 N=256 K=64        (1 CTA)
+//   op 1  kind::mxf4nvf4 block16, M=256 N=256 K=64        (CTA pair)
+//   op 2  kind::f16 (bf16),      M=128 N=256 K=16
+//   op 3  kind::f8f6f4 (E4M3),   M=128 N=256 K=32
+//   op 4  kind::i8 (s8),         M=128 N=256 K=32
+//   op 5  tcgen05.cp 32x128b.warpx4 only
+//   op 6  op 0 with 12 scale-factor copies (32x128b.warpx4) per 4 MMAs
+//   op 7  op 0 with 6 scale-factor copies (128x256b) per 4 MMAs
+//   op 8  tcgen05.st 32x32b.x32 + wait::st by 4 warps (one per lane quarter)
+//   op 9  op 0 while 4 other warps store 48 columns (x16 + x32) per 4 MMAs
+//   op 10 op 1 with 12 scale-factor copies (cta_group::2 32x128b.warpx4) per 4 MMAs
+constexpr int kProbeSmem = 16384 + 32768 + 16384 + 1024;
+
+template <bool kPair>
+__device__ __forceinline__ void probe_body(int op, int iters, unsigned long long* cycles) {
+  // every tcgen05 instruction of a kernel uses the same cta_group, so the
+  // pair kernel only runs op 1 and the single-CTA kernel every other op
+  extern __shared__ __align__(1024) uint8_t psm_raw[];
+  __shared__ uint64_t done_bar;
+  __shared__ uint32_t tbase_sh;
+  __shared__ int abort_sh;
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(psm_raw) + 1023) & ~uintptr_t(1023));
+  for (int i = threadIdx.x; i < (kProbeSmem - 1024) / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(sm)[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) { mbar_init(&done_bar, 1); abort_sh = 0; fence_mbar_init(); }
+  if (warp == 0) {
+    if constexpr (kPair) { tmem_alloc_pair(&tbase_sh, 512); tmem_relinquish_pair(); }
+    else { tmem_alloc(&tbase_sh, 512); tmem_relinquish(); }
+  }
+  tc_fence_before();
+  if constexpr (kPair) cluster_sync(); else __syncthreads();
+  tc_fence_after();
+  const uint32_t t = tbase_sh;
+  bool issuer = threadIdx.x == 0;
+  if constexpr (kPair) issuer = issuer && cluster_ctarank() == 0;
+  if (issuer) {
+    const uint32_t a = smem_u32(sm), b = a + 16384, sf = b + 32768;
+    // zero the scale-factor columns [256, 352) from zeroed shared memory
+    for (int q = 0; q < 24; ++q) {
+      if constexpr (kPair) tmem_cp_32x128b_x4_pair(t + 256 + 4 * q, desc_sf_32x16(sf + 512 * (q & 15)));
+      else tmem_cp_32x128b_x4(t + 256 + 4 * q, desc_sf_32x16(sf + 512 * (q & 15)));
+    }
+    const unsigned long long t0 = clock64();
+    for (int i = 0; i < iters; ++i) {
+      const uint32_t acc = i > 0;
+      if constexpr (kPair) {
+        if (op == 10 && (i & 3) == 0)
+          for (int q = 0; q < 12; ++q) tmem_cp_32x128b_x4_pair(t + 256 + 4 * q, desc_sf_32x16(sf + 512 * q));
+        mma_nvf4_pair(t, desc_k_sw128(a), desc_k_sw128(b), idesc_nvf4(256, 256), t + 256 + 4 * (i & 3),
+                      t + 288 + 8 * (i & 3), acc);
+      } else {
+        switch (op) {
+          case 0: mma_nvf4(t, desc_k_sw128(a), desc_k_sw128(b), idesc_nvf4(128, 256), t + 256, t + 288, acc); break;
+          case 2: mma_f16(t, desc_k_sw128(a), desc_k_sw128(b), idesc_f16_bf16(128, 256), acc); break;
+          case 3: mma_f8(t, desc_k_sw128(a), desc_k_sw128(b), idesc_f8_e4m3(128, 256), acc); break;
+          case 4: mma_i8(t, desc_k_sw128(a), desc_k_sw128(b), idesc_i8(128, 256), acc); break;
+          case 5: tmem_cp_32x128b_x4(t + 256 + 4 * (i & 15), desc_sf_32x16(sf + 512 * (i & 15))); break;
+          case 6:
+            if ((i & 3) == 0)
+              for (int q = 0; q < 12; ++q) tmem_cp_32x128b_x4(t + 256 + 4 * q, desc_sf_32x16(sf + 512 * q));
+            mma_nvf4(t, desc_k_sw128(a), desc_k_sw128(b), idesc_nvf4(128, 256), t + 256 + 4 * (i & 3),
+                     t + 288 + 8 * (i & 3), acc);
+            break;
+          case 7:
+            if ((i & 3) == 0)
+              for (int q = 0; q < 6; ++q) tmem_cp_128x256b(t + 256 + 8 * q, desc_sf_32x16(sf + 2048 * q));
+            mma_nvf4(t, desc_k_sw128(a), desc_k_sw128(b), idesc_nvf4(128, 256), t + 256 + 4 * (i & 3),
+                     t + 288 + 8 * (i & 3), acc);
+            break;
+          case 9:
+            mma_nvf4(t, desc_k_sw128(a), desc_k_sw128(b), idesc_nvf4(128, 256), t + 256, t + 288, acc);
+            break;
+          default: break;
+        }
+      }
+    }
+    if constexpr (kPair) mma_commit_pair(&done_bar, 0x3); else mma_commit(&done_bar);
+    mbar_wait(&done_bar, 0, &abort_sh);
+    cycles[blockIdx.x] = clock64() - t0;
+  }
+  if constexpr (!kPair) {
+    // TMEM stores from warps 4..7 (lane quarter warp % 4), columns [384, 432)
+    if ((op == 8 || op == 9) && warp >= 4) {
+      uint32_t r32[32], r16[16];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) r32[j] = j;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) r16[j] = j;
+      const uint32_t lane_base = t + ((uint32_t)((warp & 3) * 32) << 16);
+      const unsigned long long t0 = clock64();
+      const int n = op == 8 ? iters : iters / 4;
+      for (int i = 0; i < n; ++i) {
+        tmem_st_32cols(lane_base + 384, r32);
+        if (op == 9) tmem_st_16cols(lane_base + 416, r16);
+        tmem_st_wait();
+      }
+      if ((threadIdx.x & 31) == 0) cycles[gridDim.x * (warp - 3) + blockIdx.x] = clock64() - t0;
+    }
+  }
+  if constexpr (kPair) {
+    if (!issuer && threadIdx.x == 0) mbar_wait(&done_bar, 0, &abort_sh);
+  }
+  tc_fence_before();
+  if constexpr (kPair) cluster_sync(); else __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    if constexpr (kPair) tmem_dealloc_pair(t, 512); else tmem_dealloc(t, 512);
+  }
+}
+
+__global__ void __launch_bounds__(256, 1) tc_probe_kernel(int op, int iters, unsigned long long* cycles) {
+  probe_body<false>(op, iters, cycles);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
+    tc_probe_pair_kernel(int op, int iters, unsigned long long* cycles) {
+  probe_body<true>(op, iters, cycles);
+}
+
+// Test hook: the activation kernel's quotient (reciprocal + FMA correction)
+// next to the IEEE division, on the same inputs.
+__global__ void probe_div_kernel(const float* v, const float* d, int64_t n, float* q, float* q_ieee) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    const float dv = d[i];
+    q[i] = recip_ok(dv) ? div_by_recip(v[i], dv, __frcp_rn(dv)) : __fdiv_rn(v[i], dv);
+    q_ieee[i] = __fdiv_rn(v[i], dv);
+  }
+}
+
 }  // namespace dev
 }  // namespace svdq
 
@@ -703,6 +1029,19 @@ extern "C" svdq_status svdq_decode_act_host(const svdq_params* p, const uint8_t*
                                             uint8_t* codes, void* scales, float* u);
 
 namespace {
+
+thread_local char g_last_error[256] = "";
+
+// Record a failed CUDA call for svdq_last_error_string and return SVDQ_ERR_CUDA.
+svdq_status cuda_fail(cudaError_t e, const char* where) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, cudaGetErrorString(e), (int)e);
+  return SVDQ_ERR_CUDA;
+}
+
+svdq_status launch_status(const char* where) {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SVDQ_OK : cuda_fail(e, where);
+}
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -719,19 +1058,20 @@ bool encoder() {
 }
 
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
-              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
-  return g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Per-device capability check and one-time kernel attributes.
 struct DevState {
   bool checked = false, ok = false;
+  int sms = 0;
 };
 std::mutex g_dev_mu;
 DevState g_dev[64];
@@ -746,14 +1086,14 @@ svdq_status device_ready() {
     cudaDeviceProp prop;
     if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return SVDQ_ERR_CUDA;
     d.ok = prop.major == 10 && prop.minor == 0;
+    d.sms = prop.multiProcessorCount;
     if (d.ok) {
-      const int fp4_smem = dev::kStages * dev::kFp4StageBytes + 1024;
       const int i4_smem = dev::kStages * (dev::kI4StageBytes + dev::kI4ScaleSlot) + 1024;
-      d.ok = cudaFuncSetAttribute(dev::gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  fp4_smem) == cudaSuccess &&
+      d.ok = cudaFuncSetAttribute(dev::gemm_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  dev::kP_Smem) == cudaSuccess &&
              cudaFuncSetAttribute(dev::gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   i4_smem) == cudaSuccess;
-      const int act_smem = (dev::kActRows + 128) * dev::kActStride * 2;
+      const int act_smem = 2 * (dev::kActRows + 128) * dev::kActStride * 2;
       d.ok = d.ok &&
              cudaFuncSetAttribute(dev::act_quant_kernel<SVDQ_NVFP4, SVDQ_BF16>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, act_smem) == cudaSuccess &&
@@ -767,6 +1107,12 @@ svdq_status device_ready() {
     }
   }
   return d.ok ? SVDQ_OK : SVDQ_ERR_UNSUPPORTED;
+}
+
+int num_sms() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return (dev >= 0 && dev < 64 && g_dev[dev].sms > 0) ? g_dev[dev].sms : 148;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -785,38 +1131,36 @@ svdq_status check_params_dev(const svdq_params* p) {
 template <int FMT>
 void launch_act(const svdq_params* p, const dev::ActArgs& a, int64_t Mp, cudaStream_t stream) {
   const dim3 grid((unsigned)(Mp / dev::kActRows));
-  const size_t smem = (size_t)(dev::kActRows + p->rank) * dev::kActStride * 2;
+  const size_t smem = (size_t)2 * (dev::kActRows + p->rank) * dev::kActStride * 2;
   if (p->act_dtype == SVDQ_BF16) dev::act_quant_kernel<FMT, SVDQ_BF16><<<grid, 256, smem, stream>>>(a);
   else dev::act_quant_kernel<FMT, SVDQ_F16><<<grid, 256, smem, stream>>>(a);
 }
 
 }  // namespace
 
-extern "C" {
+namespace {
 
-svdq_status svdq_linear(const svdq_params* p, const void* blob_dev, const void* X, int64_t M, void* Y,
-                        void* workspace, size_t ws_bytes, svdq_stream stream_) {
+svdq_status common_checks(const svdq_params* p, const void* blob_dev, int64_t M, const void* workspace,
+                          size_t ws_bytes) {
   svdq_status st = check_params_dev(p);
   if (st != SVDQ_OK) return st;
-  if (M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M < 0 || M > ((int64_t)1 << 30)) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
-  if (!blob_dev || !X || !Y || !workspace) return SVDQ_ERR_INVALID_ARG;
-  if (!aligned16(blob_dev) || !aligned16(X) || !aligned16(Y) || !aligned16(workspace)) return SVDQ_ERR_ALIGNMENT;
-  if (M > (int64_t)1 << 30) return SVDQ_ERR_INVALID_ARG;
-  const WsLayout W = ws_layout(*p, M);
-  if (ws_bytes < W.total) return SVDQ_ERR_WORKSPACE;
-  st = device_ready();
-  if (st != SVDQ_OK) return st;
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!blob_dev || !workspace) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(blob_dev) || !aligned16(workspace)) return SVDQ_ERR_ALIGNMENT;
+  if (ws_bytes < ws_layout(*p, M).total) return SVDQ_ERR_WORKSPACE;
+  return device_ready();
+}
 
+svdq_status launch_quantize(const svdq_params* p, const void* blob_dev, const void* X, int64_t M,
+                            void* workspace, cudaStream_t stream) {
+  const WsLayout W = ws_layout(*p, M);
   const BlobLayout B = blob_layout(*p);
   const uint8_t* blob = static_cast<const uint8_t*>(blob_dev);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const int K = p->K, N = p->N, r = p->rank, lrw = lr_width(*p);
-
   dev::ActArgs a;
   a.X = static_cast<const uint16_t*>(X);
-  a.M = M; a.Mp = W.Mp; a.K = K; a.r = r; a.lrw = lrw; a.nseg = nseg_of(*p);
+  a.M = M; a.Mp = W.Mp; a.K = p->K; a.r = p->rank; a.lrw = lr_width(*p); a.nseg = nseg_of(*p);
   a.inv_lambda = reinterpret_cast<const float*>(blob + B.off_inv_lambda);
   a.l1t = reinterpret_cast<const uint16_t*>(blob + B.off_l1t);
   a.hdr = reinterpret_cast<const BlobHeader*>(blob);
@@ -824,11 +1168,36 @@ svdq_status svdq_linear(const svdq_params* p, const void* blob_dev, const void* 
   a.ux = reinterpret_cast<uint16_t*>(ws + W.off_ux);
   if (p->fmt == SVDQ_NVFP4) launch_act<SVDQ_NVFP4>(p, a, W.Mp, stream);
   else launch_act<SVDQ_INT4_G64>(p, a, W.Mp, stream);
-  if (cudaGetLastError() != cudaSuccess) return SVDQ_ERR_CUDA;
+  return launch_status("act_quant_kernel launch");
+}
 
-  CUtensorMap tm_a, tm_b, tm_ua, tm_ub;
+svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, void* Y, void* workspace,
+                        cudaStream_t stream) {
+  const WsLayout W = ws_layout(*p, M);
+  const BlobLayout B = blob_layout(*p);
+  const uint8_t* blob = static_cast<const uint8_t*>(blob_dev);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int K = p->K, N = p->N, r = p->rank, lrw = lr_width(*p);
   const bool fp4 = p->fmt == SVDQ_NVFP4;
-  const uint64_t krow = fp4 ? (uint64_t)K / 2 : (uint64_t)K;
+  if (fp4) {
+    dev::PairArgs g;
+    g.M = M; g.Mp = W.Mp; g.N = N; g.K = K;
+    g.lr_iters = r > 0 ? lrw / 64 : 0;
+    g.k_iters = K / 256;
+    g.atiles = ws + W.off_xq;
+    g.wtiles = blob + B.off_wq;
+    g.utiles = ws + W.off_ux;
+    g.l2tiles = blob + B.off_l2x;
+    g.bias = reinterpret_cast<const float*>(blob + B.off_bias);
+    g.hdr = reinterpret_cast<const BlobHeader*>(blob);
+    g.Y = static_cast<uint16_t*>(Y);
+    const int tiles = (N / 256) * (int)(W.Mp / 256);
+    const int pairs = std::max(1, std::min(tiles, num_sms() / 2));
+    dev::gemm_nvfp4_pair_kernel<<<2 * pairs, dev::kP_Threads, dev::kP_Smem, stream>>>(g);
+    return launch_status("gemm_nvfp4_pair_kernel launch");
+  }
+  CUtensorMap tm_a, tm_b, tm_ua, tm_ub;
+  const uint64_t krow = (uint64_t)K;
   bool ok = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + W.off_xq, krow, (uint64_t)M, krow, 128, dev::kBM) &&
             make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, blob + B.off_wq, krow, (uint64_t)N, krow, 128, dev::kBN);
   if (r > 0) {
@@ -837,14 +1206,13 @@ svdq_status svdq_linear(const svdq_params* p, const void* blob_dev, const void* 
          make_map(&tm_ub, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, blob + B.off_l2x, (uint64_t)lrw, (uint64_t)N,
                   (uint64_t)lrw * 2, 64, dev::kBN);
   } else {
-    tm_ua = tm_a; tm_ub = tm_b;   // unused
+    tm_ua = tm_a; tm_ub = tm_b;   // not read when rank is 0
   }
-  if (!ok) return SVDQ_ERR_CUDA;
-
+  if (!ok) return cuda_fail(cudaErrorInvalidValue, "tensor map encode");
   dev::GemmArgs g;
   g.M = M; g.N = N; g.K = K;
   g.lr_iters = r > 0 ? lrw / 64 : 0;
-  g.k_iters = fp4 ? K / 256 : K / 128;
+  g.k_iters = K / 128;
   g.sfa = ws + W.off_xs;
   g.sfb = blob + B.off_ws;
   g.bias = reinterpret_cast<const float*>(blob + B.off_bias);
@@ -852,15 +1220,43 @@ svdq_status svdq_linear(const svdq_params* p, const void* blob_dev, const void* 
   g.Y = static_cast<uint16_t*>(Y);
   g.Mp = W.Mp;
   const dim3 grid((unsigned)(N / dev::kBN), (unsigned)(W.Mp / dev::kBM));
-  if (fp4) {
-    dev::gemm_nvfp4_kernel<<<grid, 192, dev::kStages * dev::kFp4StageBytes + 1024, stream>>>(tm_a, tm_b, tm_ua,
-                                                                                        tm_ub, g);
-  } else {
-    dev::gemm_int4_kernel<<<grid, 320, dev::kStages * (dev::kI4StageBytes + dev::kI4ScaleSlot) + 1024, stream>>>(
-        tm_a, tm_b, tm_ua, tm_ub, g);
-  }
-  if (cudaGetLastError() != cudaSuccess) return SVDQ_ERR_CUDA;
-  return SVDQ_OK;
+  dev::gemm_int4_kernel<<<grid, 320, dev::kStages * (dev::kI4StageBytes + dev::kI4ScaleSlot) + 1024, stream>>>(
+      tm_a, tm_b, tm_ua, tm_ub, g);
+  return launch_status("gemm kernel launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+svdq_status svdq_quantize_act(const svdq_params* p, const void* blob_dev, const void* X, int64_t M,
+                              void* workspace, size_t ws_bytes, svdq_stream stream) {
+  svdq_status st = common_checks(p, blob_dev, M, workspace, ws_bytes);
+  if (st != SVDQ_OK || M == 0) return st;
+  if (!X) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X)) return SVDQ_ERR_ALIGNMENT;
+  return launch_quantize(p, blob_dev, X, M, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+svdq_status svdq_gemm(const svdq_params* p, const void* blob_dev, int64_t M, void* Y, void* workspace,
+                      size_t ws_bytes, svdq_stream stream) {
+  svdq_status st = common_checks(p, blob_dev, M, workspace, ws_bytes);
+  if (st != SVDQ_OK || M == 0) return st;
+  if (!Y) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(Y)) return SVDQ_ERR_ALIGNMENT;
+  return launch_gemm(p, blob_dev, M, Y, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+svdq_status svdq_linear(const svdq_params* p, const void* blob_dev, const void* X, int64_t M, void* Y,
+                        void* workspace, size_t ws_bytes, svdq_stream stream_) {
+  svdq_status st = common_checks(p, blob_dev, M, workspace, ws_bytes);
+  if (st != SVDQ_OK || M == 0) return st;
+  if (!X || !Y) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Y)) return SVDQ_ERR_ALIGNMENT;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  st = launch_quantize(p, blob_dev, X, M, workspace, stream);
+  if (st != SVDQ_OK) return st;
+  return launch_gemm(p, blob_dev, M, Y, workspace, stream);
 }
 
 svdq_status svdq_export_act(const svdq_params* p, const void* workspace, int64_t M, uint8_t* codes,
@@ -870,22 +1266,29 @@ svdq_status svdq_export_act(const svdq_params* p, const void* workspace, int64_t
   if (!workspace || M < 0) return SVDQ_ERR_INVALID_ARG;
   const WsLayout W = ws_layout(*p, M);
   std::vector<uint8_t> host(W.total);
-  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SVDQ_ERR_CUDA;
-  if (cudaMemcpy(host.data(), workspace, W.total, cudaMemcpyDeviceToHost) != cudaSuccess) return SVDQ_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "svdq_export_act sync");
+  e = cudaMemcpy(host.data(), workspace, W.total, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "svdq_export_act copy");
   return svdq_decode_act_host(p, host.data(), M, codes, scales, u);
 }
 
 svdq_status svdq_get_status(svdq_stream stream) {
-  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SVDQ_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "svdq_get_status sync");
   unsigned int v = 0;
-  if (cudaMemcpyFromSymbol(&v, dev::g_status, sizeof(v)) != cudaSuccess) return SVDQ_ERR_CUDA;
+  e = cudaMemcpyFromSymbol(&v, dev::g_status, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "svdq_get_status read");
   if (v != 0) {
     const unsigned int z = 0;
-    if (cudaMemcpyToSymbol(dev::g_status, &z, sizeof(z)) != cudaSuccess) return SVDQ_ERR_CUDA;
+    e = cudaMemcpyToSymbol(dev::g_status, &z, sizeof(z));
+    if (e != cudaSuccess) return cuda_fail(e, "svdq_get_status clear");
     return (svdq_status)v;
   }
   return SVDQ_OK;
 }
+
+const char* svdq_last_error_string(void) { return g_last_error; }
 
 svdq_status svdq_probe_cvt(const float* in, int64_t n, uint8_t* e2m1, uint8_t* e4m3, svdq_stream stream) {
   if (n < 0 || (n > 0 && (!in || !e2m1 || !e4m3))) return SVDQ_ERR_INVALID_ARG;
@@ -894,7 +1297,33 @@ svdq_status svdq_probe_cvt(const float* in, int64_t n, uint8_t* e2m1, uint8_t* e
   if (st != SVDQ_OK) return st;
   const int64_t blocks = (n + 255) / 256;
   dev::probe_cvt_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(in, n, e2m1, e4m3);
-  return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+  return launch_status("probe_cvt launch");
+}
+
+svdq_status svdq_probe_tc(int op, int iters, int ctas, unsigned long long* cycles, svdq_stream stream) {
+  if (op < 0 || op > 10 || iters <= 0 || ctas <= 0 || !cycles) return SVDQ_ERR_INVALID_ARG;
+  svdq_status st = device_ready();
+  if (st != SVDQ_OK) return st;
+  cudaError_t e = cudaFuncSetAttribute(dev::tc_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       dev::kProbeSmem);
+  if (e != cudaSuccess) return cuda_fail(e, "tc_probe_kernel attribute");
+  e = cudaFuncSetAttribute(dev::tc_probe_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dev::kProbeSmem);
+  if (e != cudaSuccess) return cuda_fail(e, "tc_probe_pair_kernel attribute");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (op == 1 || op == 10) dev::tc_probe_pair_kernel<<<(ctas + 1) / 2 * 2, 128, dev::kProbeSmem, s>>>(op, iters, cycles);
+  else dev::tc_probe_kernel<<<ctas, 256, dev::kProbeSmem, s>>>(op, iters, cycles);
+  return launch_status("tc_probe launch");
+}
+
+svdq_status svdq_probe_div(const float* v, const float* d, int64_t n, float* q, float* q_ieee,
+                           svdq_stream stream) {
+  if (n < 0 || (n > 0 && (!v || !d || !q || !q_ieee))) return SVDQ_ERR_INVALID_ARG;
+  if (n == 0) return SVDQ_OK;
+  svdq_status st = device_ready();
+  if (st != SVDQ_OK) return st;
+  const int64_t blocks = (n + 255) / 256;
+  dev::probe_div_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(v, d, n, q, q_ieee);
+  return launch_status("probe_div launch");
 }
 
 }  // extern "C"

@@ -30,6 +30,7 @@ svdq_status check_params(const svdq_params* p) {
   if (p->rank < 0 || p->rank > 128 || p->rank % 16 != 0 || p->rank > std::min(p->K, p->N))
     return SVDQ_ERR_INVALID_ARG;
   if (p->fmt != SVDQ_INT4_G64 && p->fmt != SVDQ_NVFP4) return SVDQ_ERR_UNSUPPORTED;
+  if (p->fmt == SVDQ_NVFP4 && p->K % 256 != 0) return SVDQ_ERR_INVALID_ARG;   // whole 256-wide K slabs
   if (p->act_dtype != SVDQ_F16 && p->act_dtype != SVDQ_BF16) return SVDQ_ERR_UNSUPPORTED;
   if (!(p->alpha >= 0.0f && p->alpha <= 1.0f)) return SVDQ_ERR_INVALID_ARG;
   if (p->smooth != 0 && p->smooth != 1) return SVDQ_ERR_INVALID_ARG;
@@ -430,6 +431,7 @@ svdq_status svdq_prepare(const svdq_params* p, const float* Wt, const float* bia
   //        output channel n along K.
   uint8_t* wq = base + L.off_wq;
   uint8_t* wsb = base + L.off_ws;
+  (void)wsb;
   std::vector<float> R((size_t)N * K);
 #pragma omp parallel for schedule(static)
   for (int n = 0; n < N; ++n)
@@ -457,13 +459,26 @@ svdq_status svdq_prepare(const svdq_params* p, const float* Wt, const float* bia
     for (size_t i = 0; i < R.size(); ++i) amax = std::max(amax, fabsf(R[i]));
     const float s_g = nvfp4_tensor_scale(amax);
     h->s_gw = s_g;
-    const int kb = K / kBlockFp4;
+    // weight tiles [n/128][slab]: swizzled codes + the scales of the tile's 256-row pair
+    const int kb = K / kBlockFp4, ksl = K / 256;
 #pragma omp parallel for schedule(static)
     for (int n = 0; n < N; ++n) {
       std::vector<uint8_t> c(K), e(kb);
       nvfp4_quant_row(&R[(size_t)n * K], K, s_g, c.data(), e.data());
-      for (int j = 0; j < K; j += 2) wq[(size_t)n * (K / 2) + j / 2] = (uint8_t)(c[j] | (c[j + 1] << 4));
-      for (int b = 0; b < kb; ++b) wsb[sf_offset(n, b, kb)] = e[b];
+      const int nb = n / 128, rr = n % 128, half = nb & 1, pb = nb & ~1;
+      for (int t = 0; t < ksl; ++t) {
+        uint8_t* tile = wq + ((size_t)nb * ksl + t) * kWTile;
+        for (int cb = 0; cb < 128; ++cb) {
+          const int j = t * 256 + 2 * cb;
+          tile[sw128(rr, cb)] = (uint8_t)(c[j] | (c[j + 1] << 4));
+        }
+        for (int b = 0; b < 16; ++b) {
+          const uint8_t sc = e[t * 16 + b];
+          // both tiles of the pair carry the pair's scales
+          for (int q = 0; q < 2; ++q)
+            wq[((size_t)(pb + q) * ksl + t) * kWTile + kTileCodes + half * 2048 + tile_sf(rr, b)] = sc;
+        }
+      }
     }
   }
 
@@ -483,13 +498,19 @@ svdq_status svdq_prepare(const svdq_params* p, const float* Wt, const float* bia
     for (int j = 0; j < K; ++j) l1t[(size_t)i * K + j] = dtype_bits(L1[(size_t)j * r + i], dt);
   uint16_t* l2x = (uint16_t*)(base + L.off_l2x);
   const int w2 = lr_width(*p);
+  // element (n, e) of the N x w2 low-rank B operand: row-major (INT4) or tiles (NVFP4)
+  auto l2x_at = [&](int n, int e) -> uint16_t& {
+    if (p->fmt != SVDQ_NVFP4) return l2x[(size_t)n * w2 + e];
+    uint8_t* tile = base + L.off_l2x + ((size_t)(n / 128) * (w2 / 64) + e / 64) * kLRTile;
+    return *reinterpret_cast<uint16_t*>(tile + sw128(n % 128, (e % 64) * 2));
+  };
   for (int n = 0; n < N; ++n)
     for (int i = 0; i < r; ++i) {
       const double v = L2[(size_t)i * N + n];
       const double hi = bf16_round(v), lo = v - hi;                  // lo exact in bf16
-      l2x[(size_t)n * w2 + i] = bf16_bits_exact(hi);
-      l2x[(size_t)n * w2 + r + i] = bf16_bits_exact(hi);
-      if (L.nseg == 3) l2x[(size_t)n * w2 + 2 * r + i] = bf16_bits_exact(lo);
+      l2x_at(n, i) = bf16_bits_exact(hi);
+      l2x_at(n, r + i) = bf16_bits_exact(hi);
+      if (L.nseg == 3) l2x_at(n, 2 * r + i) = bf16_bits_exact(lo);
     }
   float* bb = (float*)(base + L.off_bias);
   for (int n = 0; n < N; ++n) bb[n] = bias ? bias[n] : 0.0f;
@@ -540,10 +561,15 @@ svdq_status svdq_blob_export(const svdq_params* p, const void* blob, float* inv_
   if (L2) {
     const uint16_t* l2x = (const uint16_t*)(base + L.off_l2x);
     const int w2 = lr_width(*p);
+    auto at = [&](int n, int e) -> uint16_t {
+      if (p->fmt != SVDQ_NVFP4) return l2x[(size_t)n * w2 + e];
+      const uint8_t* tile = base + L.off_l2x + ((size_t)(n / 128) * (w2 / 64) + e / 64) * kLRTile;
+      return *reinterpret_cast<const uint16_t*>(tile + sw128(n % 128, (e % 64) * 2));
+    };
     for (int i = 0; i < r; ++i)
       for (int n = 0; n < N; ++n) {
-        double v = bf16_value(l2x[(size_t)n * w2 + i]);
-        if (L.nseg == 3) v += bf16_value(l2x[(size_t)n * w2 + 2 * r + i]);
+        double v = bf16_value(at(n, i));
+        if (L.nseg == 3) v += bf16_value(at(n, 2 * r + i));
         L2[(size_t)i * N + n] = dtype_bits(v, dt);
       }
   }
@@ -553,7 +579,8 @@ svdq_status svdq_blob_export(const svdq_params* p, const void* blob, float* inv_
     for (int n = 0; n < N; ++n)
       for (int j = 0; j < K; ++j) {
         if (p->fmt == SVDQ_NVFP4) {
-          const uint8_t byte = wq[(size_t)n * (K / 2) + j / 2];
+          const uint8_t* tile = wq + ((size_t)(n / 128) * (K / 256) + j / 256) * kWTile;
+          const uint8_t byte = tile[sw128(n % 128, (j % 256) / 2)];
           wcodes[(size_t)n * K + j] = (j & 1) ? (byte >> 4) : (byte & 15);
         } else {
           wcodes[(size_t)n * K + j] = (uint8_t)(int8_t)llround(e4m3_value(wq[(size_t)n * K + j]));
@@ -565,7 +592,11 @@ svdq_status svdq_blob_export(const svdq_params* p, const void* blob, float* inv_
       uint8_t* o = (uint8_t*)wscales;
       const int kb = K / kBlockFp4;
       for (int n = 0; n < N; ++n)
-        for (int b = 0; b < kb; ++b) o[(size_t)n * kb + b] = wsb[sf_offset(n, b, kb)];
+        for (int b = 0; b < kb; ++b) {
+          // read from the tile of the row's own block (its pair partner holds the same bytes)
+          const uint8_t* tile = wq + ((size_t)(n / 128) * (K / 256) + b / 16) * kWTile;
+          o[(size_t)n * kb + b] = tile[kTileCodes + ((n / 128) & 1) * 2048 + tile_sf(n % 128, b % 16)];
+        }
     } else {
       float* o = (float*)wscales;
       const float* sw = (const float*)wsb;
@@ -590,7 +621,8 @@ svdq_status svdq_decode_act_host(const svdq_params* p, const uint8_t* ws, int64_
     for (int64_t m = 0; m < M; ++m)
       for (int j = 0; j < K; ++j) {
         if (p->fmt == SVDQ_NVFP4) {
-          const uint8_t byte = ws[W.off_xq + (size_t)m * (K / 2) + j / 2];
+          const uint8_t* tile = ws + W.off_xq + ((size_t)(m / 128) * (K / 256) + j / 256) * kATile;
+          const uint8_t byte = tile[sw128((uint32_t)(m % 128), (j % 256) / 2)];
           codes[(size_t)m * K + j] = (j & 1) ? (byte >> 4) : (byte & 15);
         } else {
           codes[(size_t)m * K + j] = (uint8_t)(int8_t)llround(e4m3_value(ws[W.off_xq + (size_t)m * K + j]));
@@ -602,7 +634,10 @@ svdq_status svdq_decode_act_host(const svdq_params* p, const uint8_t* ws, int64_
       uint8_t* o = (uint8_t*)scales;
       const int kb = K / kBlockFp4;
       for (int64_t m = 0; m < M; ++m)
-        for (int b = 0; b < kb; ++b) o[(size_t)m * kb + b] = ws[W.off_xs + sf_offset(m, b, kb)];
+        for (int b = 0; b < kb; ++b) {
+          const uint8_t* tile = ws + W.off_xq + ((size_t)(m / 128) * (K / 256) + b / 16) * kATile;
+          o[(size_t)m * kb + b] = tile[kTileCodes + tile_sf((uint32_t)(m % 128), b % 16)];
+        }
     } else {
       float* o = (float*)scales;
       const float* sx = (const float*)(ws + W.off_xs);
@@ -613,10 +648,14 @@ svdq_status svdq_decode_act_host(const svdq_params* p, const uint8_t* ws, int64_
   }
   if (u) {
     const uint16_t* ux = (const uint16_t*)(ws + W.off_ux);
+    auto at = [&](int64_t m, int e) -> uint16_t {
+      if (p->fmt != SVDQ_NVFP4) return ux[(size_t)m * w2 + e];
+      const uint8_t* tile = ws + W.off_ux + ((size_t)(m / 128) * (w2 / 64) + e / 64) * kLRTile;
+      return *reinterpret_cast<const uint16_t*>(tile + sw128((uint32_t)(m % 128), (e % 64) * 2));
+    };
     for (int64_t m = 0; m < M; ++m)
       for (int i = 0; i < r; ++i)
-        u[(size_t)m * r + i] = (float)(bf16_value(ux[(size_t)m * w2 + i]) +
-                                       bf16_value(ux[(size_t)m * w2 + r + i]));
+        u[(size_t)m * r + i] = (float)(bf16_value(at(m, i)) + bf16_value(at(m, r + i)));
   }
   return SVDQ_OK;
 }

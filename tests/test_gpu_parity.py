@@ -41,6 +41,34 @@ def test_probe_cvt_matches_oracle_encoders(gpu):
     assert len(bad4) == 0, (x[bad4[:8]], g4[bad4[:8]], r4[bad4[:8]])
 
 
+def test_probe_division_matches_ieee(gpu):
+    """The activation kernel's quotient (reciprocal + FMA correction) equals
+    the IEEE round-to-nearest division on random operands and on operands
+    placed at and around the code decision points (E2M1 midpoints, INT4
+    half-integers) times the divisor."""
+    import torch
+    rng = np.random.default_rng(2)
+    n = 1 << 20
+    d = np.exp(rng.uniform(np.log(1e-37), np.log(1e30), n)).astype(np.float32)
+    t = rng.uniform(-8, 8, n)
+    marks = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.5, 1.5, 2.5, 3.5, 4.5, 5.5, 6.5, 7.0])
+    t[: n // 2] = rng.choice(marks, n // 2) * rng.choice([-1.0, 1.0], n // 2)
+    v = (t * d).astype(np.float32)
+    k = n // 4
+    v[:k] = np.nextafter(v[:k], np.float32(np.inf))
+    v[k:2 * k] = np.nextafter(v[k:2 * k], np.float32(-np.inf))
+    v[-64:] = 0.0
+    vd, dd = torch.from_numpy(v).cuda(), torch.from_numpy(d).cuda()
+    q = torch.empty_like(vd); qi = torch.empty_like(vd)
+    sv.probe_div(vd, dd, q, qi)
+    torch.cuda.synchronize()
+    a, b = q.cpu().numpy(), qi.cpu().numpy()
+    bad = np.flatnonzero(a.view(np.uint32) != b.view(np.uint32))
+    assert len(bad) == 0, (v[bad[:5]], d[bad[:5]], a[bad[:5]], b[bad[:5]])
+    # and the IEEE quotient equals the host's fp32 division
+    assert np.array_equal(b.view(np.uint32), (v / d).astype(np.float32).view(np.uint32))
+
+
 def test_tiny_int4_config(gpu):
     """The tiny INT4 layer (M=256, K=512, N=512, fp16, rank 16, 4 outlier
     channels x100): every output and every code against the oracle."""

@@ -207,6 +207,36 @@ svdq_status svdq_probe_div(const float* v, const float* d, int64_t n, float* q, 
  */
 svdq_status svdq_probe_tc(int op, int iters, int ctas, unsigned long long* cycles, svdq_stream stream);
 
+/*
+ * svdq_linear without a caller-supplied workspace: the quantised activations
+ * and the down projection go to a scratch buffer that the library holds in
+ * static device memory (SVDQ_NOALLOC_SCRATCH_BYTES per device, 256-byte
+ * aligned, part of the library's device image).  Nothing is allocated by this
+ * call: no cudaMalloc, no cudaFree, no allocating library routine.  The
+ * SVDQuant pages have no counterpart; this entry point exists for callers that
+ * must not allocate device memory at the point of the call (for example a
+ * host framework whose allocator is not reachable from where the layer runs,
+ * or code running while allocation is forbidden).
+ *
+ *   p, blob_dev, X, M, Y, stream   as for svdq_linear.
+ *
+ * Limit: the workspace that svdq_workspace_bytes(p, M) reports must fit in
+ * SVDQ_NOALLOC_SCRATCH_BYTES, otherwise the call returns SVDQ_ERR_WORKSPACE
+ * and svdq_last_error_string names both sizes; nothing is launched.  16 MiB
+ * covers, e.g., K = 3072 layers at 4608 tokens in both formats.
+ * Nothing in the scratch has to start at zero: the first kernel writes every
+ * byte that the second reads.
+ * The first call on each device performs one-time set-up with that device
+ * current (device query, kernel attributes, and the lookup of the scratch
+ * buffer's device address); make that first call before any stream capture.
+ * There is ONE scratch buffer per device: calls that may overlap on the GPU
+ * (different streams, or different host threads, without ordering between
+ * them) race on it and corrupt each other's results.  Order such calls.
+ */
+#define SVDQ_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+svdq_status svdq_linear_noalloc(const svdq_params* p, const void* blob_dev, const void* X, int64_t M,
+                                void* Y, svdq_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -63,6 +63,7 @@ def _load():
         "svdq_probe_cvt": (ctypes.c_int, [vp, i64, vp, vp, vp]),
         "svdq_probe_div": (ctypes.c_int, [vp, vp, i64, vp, vp, vp]),
         "svdq_probe_tc": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp]),
+        "svdq_linear_noalloc": (ctypes.c_int, [P, vp, vp, i64, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -73,7 +74,9 @@ def _load():
 _lib = _load()
 EXPORTED = ("svdq_blob_bytes", "svdq_prepare", "svdq_blob_check", "svdq_blob_export",
             "svdq_workspace_bytes", "svdq_linear", "svdq_quantize_act", "svdq_gemm", "svdq_export_act", "svdq_get_status",
-            "svdq_status_string", "svdq_last_error_string", "svdq_probe_cvt", "svdq_probe_div", "svdq_probe_tc")
+            "svdq_status_string", "svdq_last_error_string", "svdq_probe_cvt", "svdq_probe_div", "svdq_probe_tc",
+            "svdq_linear_noalloc")
+NOALLOC_SCRATCH_BYTES = 16 << 20   # SVDQ_NOALLOC_SCRATCH_BYTES
 
 
 def lib():
@@ -166,6 +169,15 @@ def linear(p: svdq_params, blob_dev, X, M: int, Y, workspace, stream=None):
     st = _lib.svdq_linear(ctypes.byref(p), _ptr(blob_dev), _ptr(X), M, _ptr(Y), _ptr(workspace),
                           workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "svdq_linear")
+
+
+def linear_noalloc(p: svdq_params, blob_dev, X, M: int, Y, stream=None):
+    """svdq_linear with the library's static scratch as workspace (allocates
+    nothing; calls on one device must not overlap)."""
+    st = _lib.svdq_linear_noalloc(ctypes.byref(p), _ptr(blob_dev), _ptr(X), M, _ptr(Y), _stream(stream))
+    if st == ERR_WORKSPACE:
+        raise SVDQError(st, "svdq_linear_noalloc: " + _lib.svdq_last_error_string().decode())
+    _check(st, "svdq_linear_noalloc")
 
 
 def quantize_act(p: svdq_params, blob_dev, X, M: int, workspace, stream=None):

@@ -1327,3 +1327,57 @@ svdq_status svdq_probe_div(const float* v, const float* d, int64_t n, float* q, 
 }
 
 }  // extern "C"
+
+// ======================================================================= allocation-free entry point
+// Some callers cannot allocate device memory where the layer runs (their
+// allocator is out of reach there, or allocation is forbidden at that point),
+// so this entry point takes its workspace from a buffer in the library's own
+// static device memory instead of from the caller.  One buffer per device;
+// overlapping calls on one device share it.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SVDQ_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64] = {};
+
+// Device address of the static scratch on the current device, looked up once
+// per device (with that device current) and cached.
+svdq_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "svdq_linear_noalloc cudaGetDevice");
+  if (dev < 0 || dev >= 64) return SVDQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* a = nullptr;
+    e = cudaGetSymbolAddress(&a, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "svdq_linear_noalloc cudaGetSymbolAddress");
+    g_scratch_addr[dev] = a;
+  }
+  *out = g_scratch_addr[dev];
+  return SVDQ_OK;
+}
+
+}  // namespace
+
+extern "C" svdq_status svdq_linear_noalloc(const svdq_params* p, const void* blob_dev, const void* X, int64_t M,
+                                           void* Y, svdq_stream stream) {
+  svdq_status st = check_params_dev(p);
+  if (st != SVDQ_OK) return st;
+  if (M < 0 || M > ((int64_t)1 << 30)) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  const size_t need = ws_layout(*p, M).total;
+  if (need > SVDQ_NOALLOC_SCRATCH_BYTES) {
+    snprintf(g_last_error, sizeof(g_last_error),
+             "svdq_linear_noalloc: workspace of %zu bytes exceeds the static scratch of %zu bytes", need,
+             (size_t)SVDQ_NOALLOC_SCRATCH_BYTES);
+    return SVDQ_ERR_WORKSPACE;
+  }
+  st = device_ready();
+  if (st != SVDQ_OK) return st;
+  void* ws = nullptr;
+  st = noalloc_scratch(&ws);
+  if (st != SVDQ_OK) return st;
+  return svdq_linear(p, blob_dev, X, M, Y, ws, SVDQ_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -153,8 +153,13 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Arrive on an mbarrier of a CTA of this cluster (default semantics:
+// release at CTA scope).  Callers order their tensor-memory work before it
+// with tcgen05.wait + tcgen05.fence::before_thread_sync.  A cluster-scope
+// release here waits for this SM's outstanding bulk copies to land, which
+// serialises the load ring: measured 3x slower on a pair ring of 38 KB stages.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
 __device__ __forceinline__ void st_cluster_u32(uint32_t addr_cluster, uint32_t v) {

@@ -442,7 +442,8 @@ constexpr int kS_Size = kATile + kWTile;           // 38912
 constexpr int kP_Stages = 5;
 constexpr int kEpiWarps = 8;
 constexpr int kP_Threads = 16 * 32;
-constexpr int kP_Smem = kP_Stages * kS_Size + kEpiWarps * 128 * 4 + 1024;
+constexpr int kEpiChunk = 32 * 128;               // 32 rows x 64 bf16 columns, 128-byte swizzled
+constexpr int kP_Smem = kP_Stages * kS_Size + kEpiWarps * kEpiChunk + 1024;
 
 struct PairArgs {
   int64_t M, Mp;
@@ -459,14 +460,14 @@ struct PairArgs {
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
-    gemm_nvfp4_pair_kernel(const PairArgs g) {
+    gemm_nvfp4_pair_kernel(const PairArgs g, const __grid_constant__ CUtensorMap tm_y) {
   extern __shared__ __align__(1024) uint8_t gsmem_raw[];
   __shared__ uint64_t landed_bar[kP_Stages], empty_bar[kP_Stages], ready_bar[kP_Stages], accf_bar, acce_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
-  float* bias_smem = reinterpret_cast<float*>(smem + kP_Stages * kS_Size);
+  uint8_t* ychunks = smem + kP_Stages * kS_Size;   // one 4 KB output chunk per epilogue warp
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -597,19 +598,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
     }
   } else {
     regs_inc<184>();
-    // epilogue warps 8..15 (both CTAs)
+    // epilogue warps 8..15 (both CTAs): TMEM -> registers, release TMEM,
+    // then y = alpha * acc + bias -> bf16, written through a swizzled 4 KB
+    // shared-memory chunk (32 rows x 64 columns) by TMA stores, so that
+    // global writes are whole 128-byte row segments.
     const int q = warp & 3;
     const int h = (warp - 8) >> 2;
     const uint32_t taddr = tbase + ((uint32_t)(q * 32) << 16) + h * 128;
     const uint32_t acce_leader = mapa_shared(smem_u32(&acce_bar), 0);
     const float alpha = g.hdr->s_gx * g.hdr->s_gw;
-    float* bsm = bias_smem + (warp - 8) * 128;
+    uint8_t* ybuf = ychunks + (warp - 8) * kEpiChunk;
     int tcount = 0;
     for (int tile = pair; tile < num_tiles; tile += pairs, ++tcount) {
       const int mt = tile / n_tiles, nt = tile % n_tiles;
       const int col0 = nt * 256 + h * 128;
-      *reinterpret_cast<float4*>(bsm + lane * 4) = __ldg(reinterpret_cast<const float4*>(g.bias + col0 + lane * 4));
-      __syncwarp();
+      float bl[4];   // bias of columns col0 + 32 j + lane
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bl[j] = __ldg(g.bias + col0 + 32 * j + lane);
       if (!mbar_wait(&accf_bar, tcount & 1, abort_flag)) { give_up_both(); break; }
       tc_fence_after();
       uint32_t v[128];
@@ -621,24 +626,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acce_leader);
-      const int64_t m = (int64_t)mt * 256 + 128 * rank + q * 32 + lane;
-      if (m < g.M) {
-        uint4* dst = reinterpret_cast<uint4*>(g.Y + (size_t)m * g.N + col0);
+      const int64_t row0 = (int64_t)mt * 256 + 128 * rank + q * 32;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+      for (int k = 0; k < 2; ++k) {
+        uint4 pk[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const int e = c * 8 + 2 * j;
-            const float y0 = fmaf(alpha, __uint_as_float(v[e]), bsm[e]);
-            const float y1 = fmaf(alpha, __uint_as_float(v[e + 1]), bsm[e + 1]);
+            const int e = 64 * k + 8 * c + 2 * j;
+            const float b0 = __shfl_sync(0xffffffffu, bl[e >> 5], e & 31);
+            const float b1 = __shfl_sync(0xffffffffu, bl[(e + 1) >> 5], (e + 1) & 31);
+            const float y0 = fmaf(alpha, __uint_as_float(v[e]), b0);
+            const float y1 = fmaf(alpha, __uint_as_float(v[e + 1]), b1);
             w[j] = (uint32_t)bf16_rn(y0) | ((uint32_t)bf16_rn(y1) << 16);
           }
-          dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+          pk[c] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        // the chunk buffer is free once the previous TMA store has read it
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(ybuf + lane * 128 + ((c ^ (lane & 7)) << 4)) = pk[c];
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < g.M) {
+          tma_store_2d(&tm_y, ybuf, col0 + 64 * k, (int)row0);
+          bulk_commit();
         }
       }
-      __syncwarp();
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -1191,9 +1212,12 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
     g.bias = reinterpret_cast<const float*>(blob + B.off_bias);
     g.hdr = reinterpret_cast<const BlobHeader*>(blob);
     g.Y = static_cast<uint16_t*>(Y);
+    CUtensorMap tm_y;
+    if (!make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 64, 32))
+      return cuda_fail(cudaErrorInvalidValue, "tensor map encode (Y)");
     const int tiles = (N / 256) * (int)(W.Mp / 256);
     const int pairs = std::max(1, std::min(tiles, num_sms() / 2));
-    dev::gemm_nvfp4_pair_kernel<<<2 * pairs, dev::kP_Threads, dev::kP_Smem, stream>>>(g);
+    dev::gemm_nvfp4_pair_kernel<<<2 * pairs, dev::kP_Threads, dev::kP_Smem, stream>>>(g, tm_y);
     return launch_status("gemm_nvfp4_pair_kernel launch");
   }
   CUtensorMap tm_a, tm_b, tm_ua, tm_ub;

@@ -334,16 +334,18 @@ def main():
     assert sv.get_status() == sv.OK
 
     peaks = measured_peaks()
-    if peaks and "bf16_tflops_sustained" in peaks:
-        peak = float(peaks["bf16_tflops_sustained"]) * (NOMINAL_FP4_TFLOPS / NOMINAL_BF16_TFLOPS)
-        peak_note = ("of measured: sustained cuBLAS bf16 "
-                     f"{peaks['bf16_tflops_sustained']} TFLOP/s x 4 (nominal dense FP4/BF16 ratio)")
+    # The timed loop lasts tens of milliseconds at full clocks, so the GEMM is
+    # compared with the burst (not the power-capped sustained) cuBLAS figure.
+    if peaks and "bf16_tflops" in peaks:
+        peak = float(peaks["bf16_tflops"]) * (NOMINAL_FP4_TFLOPS / NOMINAL_BF16_TFLOPS)
+        peak_note = ("of measured: burst cuBLAS bf16 "
+                     f"{peaks['bf16_tflops']} TFLOP/s x 4 (nominal dense FP4/BF16 ratio)")
     else:
-        peak = 1400.0 * 4
-        peak_note = "of fallback: 1.4 PFLOP/s sustained bf16 x 4"
+        peak = 1590.0 * 4
+        peak_note = "of fallback: 1.59 PFLOP/s burst bf16 x 4"
     gemm_flops = flops(M, K, N, r)
     achieved = gemm_flops / (ms_gemm * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "gemm_nvfp4_kernel", "achieved": achieved, "peak": peak,
+    roofline = {"bound": "tensor", "kernel": "gemm_nvfp4_pair_kernel", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None, "peak_source": peak_note,
                 "frac_of_nominal_fp4": achieved / NOMINAL_FP4_TFLOPS,
                 "alg_flops_per_launch": gemm_flops,

@@ -87,7 +87,9 @@ struct ActArgs {
   uint16_t* ux;
 };
 
-constexpr int kActRows = 16;     // tokens per CTA
+constexpr int kActRows = 32;     // tokens per CTA
+constexpr int kActThreads = 512;
+constexpr int kActSmemMax = 232448;
 constexpr int kActChunk = 256;   // K elements per step
 constexpr int kActStride = kActChunk + 8;  // padded smem row (bf16/fp16 elements)
 
@@ -112,6 +114,14 @@ __device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// Number of L1^T chunk buffers the activation kernel keeps in shared memory
+// (3 lets the copies run two chunks ahead; rank 128 only fits 2).
+SVDQ_HD inline int act_l1_bufs(int r) {
+  return (2 * kActRows + 3 * r) * kActStride * 2 <= kActSmemMax ? 3 : 2;
+}
+SVDQ_HD inline int act_smem_bytes(int r) { return (2 * kActRows + act_l1_bufs(r) * r) * kActStride * 2; }
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& a0, uint32_t& a1, uint32_t& a2,
                                             uint32_t& a3) {
@@ -218,17 +228,19 @@ __device__ __forceinline__ void quantize16(const float (&xh)[16], int64_t m, int
   }
 }
 
-// One CTA = 16 tokens x all of K, 8 warps.  Per 256-wide chunk, warp w owns
+// One CTA = 32 tokens x all of K, 16 warps.  Per 256-wide chunk, warp w owns
 // tokens 2w (lanes 0-15) and 2w+1 (lanes 16-31); lane l owns elements
-// 16(l%16) .. 16(l%16)+15 (two 16-byte loads).  The next chunk's loads are
-// issued before the current chunk is processed; the X^16 and L1 tiles in
-// shared memory are double-buffered so a chunk costs one __syncthreads.  The
-// down projection u = X^16 L1 runs on mma.sync (m16n8k16, fp32 accumulate),
-// one n8 tile of u per warp.
+// 16(l%16) .. 16(l%16)+15 (two 16-byte loads).  X loads run two chunks ahead
+// in registers; the L1^T chunks arrive by cp.async into a ring of 3 (2 at
+// rank 128) shared buffers, issued two (one) chunks ahead; the X^16 tile is
+// double-buffered, so a chunk costs one __syncthreads.  The down projection
+// u = X^16 L1 runs on mma.sync (m16n8k16, fp32 accumulate): 2 x r/8 tiles of
+// 16 tokens x 8 ranks, tile t on warp t % 16.
 template <int FMT, int DT>
-__global__ void __launch_bounds__(256) act_quant_kernel(const ActArgs a) {
+__global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs a) {
   extern __shared__ __align__(16) uint16_t act_smem[];
   const int K = a.K, r = a.r;
+  const int nbuf = act_l1_bufs(r), lead = nbuf - 1;
   uint16_t* const xs16_base = act_smem;
   uint16_t* const l1s_base = act_smem + 2 * kActRows * kActStride;
   auto xs16 = [&](int b) { return xs16_base + b * kActRows * kActStride; };
@@ -240,7 +252,7 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const ActArgs a) {
   const float six_sg = __fmul_rn(6.0f, s_gx);
   const float r6 = recip_ok(six_sg) ? __frcp_rn(six_sg) : 0.0f;
   const float inv_alpha = FMT == SVDQ_NVFP4 ? 1.0f / (a.hdr->s_gx * a.hdr->s_gw) : 1.0f;
-  const int n_tiles = r / 8;   // one m16 tile (16 tokens) x r/8 n8 tiles
+  const int n_mma = 2 * (r / 8);   // (16-token, 8-rank) tiles of u
 
   float acc[2][4];
 #pragma unroll
@@ -253,29 +265,37 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const ActArgs a) {
   const int col = (lane & 15) * 16;          // element offset inside the chunk
   const bool live = m < a.M;
   const uint16_t* xrow = a.X + (live ? m : 0) * K + col;
-  uint4 xc[2], xn[2];
-  xc[0] = live ? __ldg(reinterpret_cast<const uint4*>(xrow)) : make_uint4(0, 0, 0, 0);
-  xc[1] = live ? __ldg(reinterpret_cast<const uint4*>(xrow + 8)) : make_uint4(0, 0, 0, 0);
+  const int nchunks = K / kActChunk;
+  auto load_x = [&](int c, uint4 (&x)[2]) {
+    if (live && c < nchunks) {
+      x[0] = __ldg(reinterpret_cast<const uint4*>(xrow + c * kActChunk));
+      x[1] = __ldg(reinterpret_cast<const uint4*>(xrow + c * kActChunk + 8));
+    } else {
+      x[0] = make_uint4(0, 0, 0, 0);
+      x[1] = make_uint4(0, 0, 0, 0);
+    }
+  };
+  uint4 xc[2], xn[2], xnn[2];
+  load_x(0, xc);
+  load_x(1, xn);
 
-  // L1^T chunks arrive by cp.async one chunk ahead (issued right after the
-  // chunk barrier, when the other buffer is no longer read)
-  auto stage_l1 = [&](int chunk, int b) {
-    for (int idx = tid; idx < r * (kActChunk / 8); idx += 256) {
-      const int i = idx / (kActChunk / 8), c8 = idx % (kActChunk / 8);
-      cp_async_16(l1sb(b) + i * kActStride + c8 * 8, a.l1t + (size_t)i * K + chunk * kActChunk + c8 * 8);
+  // one cp.async group per chunk (empty past the end, so the counts stay uniform)
+  auto stage_l1 = [&](int chunk) {
+    if (chunk < nchunks) {
+      uint16_t* dst = l1sb(chunk % nbuf);
+      for (int idx = tid; idx < r * (kActChunk / 8); idx += kActThreads) {
+        const int i = idx / (kActChunk / 8), c8 = idx % (kActChunk / 8);
+        cp_async_16(dst + i * kActStride + c8 * 8, a.l1t + (size_t)i * K + chunk * kActChunk + c8 * 8);
+      }
     }
     cp_async_commit();
   };
-  stage_l1(0, 0);
+  for (int c = 0; c < lead; ++c) stage_l1(c);
 
-  const int nchunks = K / kActChunk;
   for (int c = 0; c < nchunks; ++c) {
     const int k0 = c * kActChunk;
     const int buf = c & 1;
-    if (c + 1 < nchunks) {
-      xn[0] = live ? __ldg(reinterpret_cast<const uint4*>(xrow + k0 + kActChunk)) : make_uint4(0, 0, 0, 0);
-      xn[1] = live ? __ldg(reinterpret_cast<const uint4*>(xrow + k0 + kActChunk + 8)) : make_uint4(0, 0, 0, 0);
-    }
+    load_x(c + 2, xnn);
     const int kk = k0 + col;
     float il[16];
 #pragma unroll
@@ -296,15 +316,19 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const ActArgs a) {
     uint4* dst = reinterpret_cast<uint4*>(xs16(buf) + rw * kActStride + col);
     dst[0] = o0;
     dst[1] = o1;
-    cp_async_wait_all();
+    // this chunk's L1^T group is complete once at most lead-1 newer ones remain
+    if (lead == 2) cp_async_wait_1(); else cp_async_wait_all();
     __syncthreads();
-    if (c + 1 < nchunks) stage_l1(c + 1, buf ^ 1);
+    // the buffer refilled here was last read by the previous chunk's MMAs
+    stage_l1(c + lead);
+    const uint16_t* l1c = l1sb(c % nbuf);
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-      const int nt = warp + 8 * t;
-      if (nt < n_tiles) {
-        const uint32_t a_base = smem_u32(xs16(buf) + (lane & 15) * kActStride + (lane >> 4) * 8);
-        const uint32_t b_base = smem_u32(l1sb(buf) + (nt * 8 + (lane & 7)) * kActStride + ((lane >> 3) & 1) * 8);
+      const int tt = warp + 16 * t;
+      if (tt < n_mma) {
+        const int mt = tt & 1, nt = tt >> 1;
+        const uint32_t a_base = smem_u32(xs16(buf) + (mt * 16 + (lane & 15)) * kActStride + (lane >> 4) * 8);
+        const uint32_t b_base = smem_u32(l1c + (nt * 8 + (lane & 7)) * kActStride + ((lane >> 3) & 1) * 8);
 #pragma unroll 4
         for (int ks = 0; ks < kActChunk / 16; ++ks) {
           uint32_t a0, a1, a2, a3, b0, b1;
@@ -314,10 +338,10 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const ActArgs a) {
         }
       }
     }
-    xc[0] = xn[0];
-    xc[1] = xn[1];
+    xc[0] = xn[0]; xc[1] = xn[1];
+    xn[0] = xnn[0]; xn[1] = xnn[1];
   }
-
+  cp_async_wait_all();
   // u' = u * inv_alpha, split into bf16 hi + lo: [hi | lo (| hi) | 0 pad];
   // NVFP4 keeps it as swizzled low-rank tiles over the padded rows
   const int64_t u_rows = FMT == SVDQ_NVFP4 ? a.Mp : a.M;
@@ -331,12 +355,13 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const ActArgs a) {
   };
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    const int nt = warp + 8 * t;
-    if (nt < n_tiles) {
+    const int tt = warp + 16 * t;
+    if (tt < n_mma) {
+      const int mt = tt & 1, nt = tt >> 1;
       const int ucol = nt * 8 + 2 * (lane & 3);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        const int64_t mu = m0 + (lane >> 2) + half * 8;
+        const int64_t mu = m0 + mt * 16 + (lane >> 2) + half * 8;
         if (mu < u_rows) {
           uint16_t hi[2], lo[2];
 #pragma unroll
@@ -355,7 +380,7 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const ActArgs a) {
   const int used = a.nseg * r;
   const int pad = a.lrw - used;
   if (pad > 0) {
-    for (int idx = tid; idx < kActRows * (pad / 2); idx += 256) {
+    for (int idx = tid; idx < kActRows * (pad / 2); idx += kActThreads) {
       const int64_t mu = m0 + idx / (pad / 2);
       if (mu < u_rows) *ux_at(mu, used + 2 * (idx % (pad / 2))) = 0;
     }
@@ -1114,7 +1139,7 @@ svdq_status device_ready() {
                                   dev::kP_Smem) == cudaSuccess &&
              cudaFuncSetAttribute(dev::gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   i4_smem) == cudaSuccess;
-      const int act_smem = 2 * (dev::kActRows + 128) * dev::kActStride * 2;
+      const int act_smem = dev::kActSmemMax;
       d.ok = d.ok &&
              cudaFuncSetAttribute(dev::act_quant_kernel<SVDQ_NVFP4, SVDQ_BF16>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, act_smem) == cudaSuccess &&
@@ -1152,9 +1177,9 @@ svdq_status check_params_dev(const svdq_params* p) {
 template <int FMT>
 void launch_act(const svdq_params* p, const dev::ActArgs& a, int64_t Mp, cudaStream_t stream) {
   const dim3 grid((unsigned)(Mp / dev::kActRows));
-  const size_t smem = (size_t)2 * (dev::kActRows + p->rank) * dev::kActStride * 2;
-  if (p->act_dtype == SVDQ_BF16) dev::act_quant_kernel<FMT, SVDQ_BF16><<<grid, 256, smem, stream>>>(a);
-  else dev::act_quant_kernel<FMT, SVDQ_F16><<<grid, 256, smem, stream>>>(a);
+  const size_t smem = (size_t)dev::act_smem_bytes(p->rank);
+  if (p->act_dtype == SVDQ_BF16) dev::act_quant_kernel<FMT, SVDQ_BF16><<<grid, dev::kActThreads, smem, stream>>>(a);
+  else dev::act_quant_kernel<FMT, SVDQ_F16><<<grid, dev::kActThreads, smem, stream>>>(a);
 }
 
 }  // namespace

@@ -166,6 +166,27 @@ def cpu_baseline(wl, ref, min_seconds=10.0):
             "sample": f"whole layer ({wl.M} tokens) x {reps} repetitions, {dt:.2f} s each, float64 numpy/BLAS"}
 
 
+def replica_batch(wl, rank):
+    """Token batch of replica `rank`: rank 0 keeps the workload's own X, every
+    other rank draws its own seeded batch of the same shape and outlier model
+    (weak scaling: one independent batch per GPU, same layer)."""
+    import synth
+    if rank == 0:
+        return wl.X
+    n_out = max(1, round(0.01 * wl.K))
+    return synth.make_x(rank, wl.M, wl.K, wl.dtype, n_out, 50.0, info={})
+
+
+def max_over_ranks(value, dist, device):
+    """Largest `value` over all ranks (the job's time is its slowest rank)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def config_dict(wl, extra=None):
     d = {"workload": f"{WORKLOAD}: FLUX.1-like FFN up projection M={wl.M} K={wl.K} N={wl.N} rank={wl.rank} "
                      f"NVFP4 (E2M1, E4M3/16, fp32 tensor scale), bf16 X, 1% outlier channels x50",
@@ -239,9 +260,7 @@ def main():
             dist.barrier()
 
     wl = synth.make_workload(WORKLOAD, seed=0)
-    if rank > 0:   # each replica gets its own token batch (same layer)
-        info = {}
-        wl.X = synth.make_x(rank, wl.M, wl.K, wl.dtype, 31, 50.0, info=info)
+    wl.X = replica_batch(wl, rank)
     p = sv.params(wl.K, wl.N, wl.rank, wl.fmt, wl.dtype, wl.alpha, wl.smooth)
     blob_host, _ = sv.prepare(p, wl.Wt, wl.bias, wl.X)
     dev = torch.device("cuda", local)
@@ -289,11 +308,7 @@ def main():
     st = sv.get_status()
     assert st == sv.OK, sv.status_string(st)
 
-    total_ms = float(sum(ms))
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(sum(ms)), dist, dev)
     ms_per_step = total_ms / args.steps
     value = flops(M, K, N, r) * world / (ms_per_step * 1e-3) / 1e12
 
@@ -325,11 +340,7 @@ def main():
     torch.cuda.synchronize()
     barrier()
     e_ms = timed(e2e_step, esteps)
-    e_total = float(sum(e_ms))
-    if dist is not None:
-        t = torch.tensor([e_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_total = float(t.item())
+    e_total = max_over_ranks(float(sum(e_ms)), dist, dev)
     e2e_value = flops(M, K, N, r) * world / (e_total / esteps * 1e-3) / 1e12
     assert sv.get_status() == sv.OK
 

@@ -52,6 +52,33 @@ def gemm_alg_bytes(M, K, N, r, fmt):
     return xq + M * 2 * r * 2 + wq + N * 2 * r * 2 + N * 4 + M * N * 2
 
 
+DEVICE_SOURCES = ("rank_gemm_svdq_b200/csrc/svdq_device.cu", "rank_gemm_svdq_b200/csrc/ptx.cuh",
+                  "rank_gemm_svdq_b200/csrc/layout.h", "include/svdq.h")
+GEMM_PROFILE = "profiles/gemm_nvfp4_pair_kernel_flux_ffn_up.md"
+
+
+def profiled_traffic():
+    """DRAM bytes per GEMM launch from the committed ncu summary, or None when
+    the device sources changed since that capture (its source_sha256)."""
+    import hashlib
+    try:
+        h = hashlib.sha256()
+        for f in DEVICE_SOURCES:
+            with open(os.path.join(ROOT, f), "rb") as fh:
+                h.update(fh.read())
+        fields = {}
+        with open(os.path.join(ROOT, GEMM_PROFILE)) as fh:
+            for line in fh:
+                if ":" in line and line.split(":")[0] in ("traffic_bytes_per_launch", "source_sha256"):
+                    k, v = line.split(":", 1)
+                    fields[k] = v.strip()
+        if fields.get("source_sha256") == h.hexdigest():
+            return int(fields["traffic_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -357,7 +384,7 @@ def main():
     gemm_flops = flops(M, K, N, r)
     achieved = gemm_flops / (ms_gemm * 1e-3) / 1e12
     roofline = {"bound": "tensor", "kernel": "gemm_nvfp4_pair_kernel", "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None, "peak_source": peak_note,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": profiled_traffic(), "peak_source": peak_note,
                 "frac_of_nominal_fp4": achieved / NOMINAL_FP4_TFLOPS,
                 "alg_flops_per_launch": gemm_flops,
                 "alg_bytes_per_launch": gemm_alg_bytes(M, K, N, r, "nvfp4"),

@@ -85,6 +85,7 @@ struct ActArgs {
   uint8_t* xq;
   uint8_t* xs;
   uint16_t* ux;
+  int ks;   // K split: a cluster of ks CTAs shares one group of 32 tokens
 };
 
 constexpr int kActRows = 32;     // tokens per CTA
@@ -228,7 +229,9 @@ __device__ __forceinline__ void quantize16(const float (&xh)[16], int64_t m, int
   }
 }
 
-// One CTA = 32 tokens x all of K, 16 warps.  Per 256-wide chunk, warp w owns
+// One CTA = 32 tokens x K / ks, 16 warps (with ks > 1 the ks CTAs of a
+// cluster split K and CTA 0 adds their partial down projections in rank
+// order through distributed shared memory, so u is deterministic).  Per 256-wide chunk, warp w owns
 // tokens 2w (lanes 0-15) and 2w+1 (lanes 16-31); lane l owns elements
 // 16(l%16) .. 16(l%16)+15 (two 16-byte loads).  X loads run two chunks ahead
 // in registers; the L1^T chunks arrive by cp.async into a ring of 3 (2 at
@@ -247,7 +250,9 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
   auto l1sb = [&](int b) { return l1s_base + b * r * kActStride; };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t m0 = (int64_t)blockIdx.x * kActRows;
+  const int KS = a.ks;
+  const int kidx = KS > 1 ? (int)cluster_ctarank() : 0;
+  const int64_t m0 = (int64_t)(blockIdx.x / KS) * kActRows;
   const float s_gx = a.hdr->s_gx;
   const float six_sg = __fmul_rn(6.0f, s_gx);
   const float r6 = recip_ok(six_sg) ? __frcp_rn(six_sg) : 0.0f;
@@ -265,9 +270,11 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
   const int col = (lane & 15) * 16;          // element offset inside the chunk
   const bool live = m < a.M;
   const uint16_t* xrow = a.X + (live ? m : 0) * K + col;
-  const int nchunks = K / kActChunk;
+  const int cpk = K / kActChunk / KS;      // chunks of this CTA: [c0, c0 + cpk)
+  const int c0 = kidx * cpk;
   auto load_x = [&](int c, uint4 (&x)[2]) {
-    if (live && c < nchunks) {
+    if (live && c < cpk) {
+      c += c0;
       x[0] = __ldg(reinterpret_cast<const uint4*>(xrow + c * kActChunk));
       x[1] = __ldg(reinterpret_cast<const uint4*>(xrow + c * kActChunk + 8));
     } else {
@@ -281,19 +288,19 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
 
   // one cp.async group per chunk (empty past the end, so the counts stay uniform)
   auto stage_l1 = [&](int chunk) {
-    if (chunk < nchunks) {
+    if (chunk < cpk) {
       uint16_t* dst = l1sb(chunk % nbuf);
       for (int idx = tid; idx < r * (kActChunk / 8); idx += kActThreads) {
         const int i = idx / (kActChunk / 8), c8 = idx % (kActChunk / 8);
-        cp_async_16(dst + i * kActStride + c8 * 8, a.l1t + (size_t)i * K + chunk * kActChunk + c8 * 8);
+        cp_async_16(dst + i * kActStride + c8 * 8, a.l1t + (size_t)i * K + (c0 + chunk) * kActChunk + c8 * 8);
       }
     }
     cp_async_commit();
   };
   for (int c = 0; c < lead; ++c) stage_l1(c);
 
-  for (int c = 0; c < nchunks; ++c) {
-    const int k0 = c * kActChunk;
+  for (int c = 0; c < cpk; ++c) {
+    const int k0 = (c0 + c) * kActChunk;
     const int buf = c & 1;
     load_x(c + 2, xnn);
     const int kk = k0 + col;
@@ -342,6 +349,33 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
     xn[0] = xnn[0]; xn[1] = xnn[1];
   }
   cp_async_wait_all();
+  if (KS > 1) {
+    // partial u of this CTA -> its shared memory; CTA 0 adds ranks 1..ks-1 in order
+    float* red = reinterpret_cast<float*>(act_smem);
+    __syncthreads();   // the last chunk's MMAs have read their operands
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int tt = warp + 16 * t;
+      if (tt < n_mma)
+        *reinterpret_cast<float4*>(red + (tt * 32 + lane) * 4) = make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
+    }
+    cluster_sync();
+    if (kidx == 0) {
+      for (int src = 1; src < KS; ++src) {
+        const uint32_t base = mapa_shared(smem_u32(red), (uint32_t)src);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const int tt = warp + 16 * t;
+          if (tt < n_mma) {
+            const float4 v = ld_cluster_f32x4(base + (uint32_t)((tt * 32 + lane) * 16));
+            acc[t][0] += v.x; acc[t][1] += v.y; acc[t][2] += v.z; acc[t][3] += v.w;
+          }
+        }
+      }
+    }
+    cluster_sync();   // every partial stays in place until CTA 0 has read it
+    if (kidx != 0) return;
+  }
   // u' = u * inv_alpha, split into bf16 hi + lo: [hi | lo (| hi) | 0 pad];
   // NVFP4 keeps it as swizzled low-rank tiles over the padded rows
   const int64_t u_rows = FMT == SVDQ_NVFP4 ? a.Mp : a.M;
@@ -1174,12 +1208,33 @@ svdq_status check_params_dev(const svdq_params* p) {
   return SVDQ_OK;
 }
 
+// K split of the activation kernel: with few 32-token groups, clusters of
+// ks CTAs share a group's K range so that more SMs work (ks | K / 256, ks <= 8).
+int act_k_split(int64_t Mp, int K) {
+  const int64_t groups = Mp / dev::kActRows;
+  const int chunks = K / dev::kActChunk;
+  int ks = 1;
+  while (ks < 8 && groups * ks * 2 <= num_sms() && chunks % (ks * 2) == 0) ks *= 2;
+  return ks;
+}
+
 template <int FMT>
-void launch_act(const svdq_params* p, const dev::ActArgs& a, int64_t Mp, cudaStream_t stream) {
-  const dim3 grid((unsigned)(Mp / dev::kActRows));
-  const size_t smem = (size_t)dev::act_smem_bytes(p->rank);
-  if (p->act_dtype == SVDQ_BF16) dev::act_quant_kernel<FMT, SVDQ_BF16><<<grid, dev::kActThreads, smem, stream>>>(a);
-  else dev::act_quant_kernel<FMT, SVDQ_F16><<<grid, dev::kActThreads, smem, stream>>>(a);
+cudaError_t launch_act(const svdq_params* p, dev::ActArgs a, int64_t Mp, cudaStream_t stream) {
+  a.ks = act_k_split(Mp, p->K);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(Mp / dev::kActRows * a.ks));
+  cfg.blockDim = dim3(dev::kActThreads);
+  cfg.dynamicSmemBytes = (size_t)dev::act_smem_bytes(p->rank);
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)a.ks;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  if (p->act_dtype == SVDQ_BF16) return cudaLaunchKernelEx(&cfg, dev::act_quant_kernel<FMT, SVDQ_BF16>, a);
+  return cudaLaunchKernelEx(&cfg, dev::act_quant_kernel<FMT, SVDQ_F16>, a);
 }
 
 }  // namespace
@@ -1212,8 +1267,9 @@ svdq_status launch_quantize(const svdq_params* p, const void* blob_dev, const vo
   a.hdr = reinterpret_cast<const BlobHeader*>(blob);
   a.xq = ws + W.off_xq; a.xs = ws + W.off_xs;
   a.ux = reinterpret_cast<uint16_t*>(ws + W.off_ux);
-  if (p->fmt == SVDQ_NVFP4) launch_act<SVDQ_NVFP4>(p, a, W.Mp, stream);
-  else launch_act<SVDQ_INT4_G64>(p, a, W.Mp, stream);
+  const cudaError_t e = p->fmt == SVDQ_NVFP4 ? launch_act<SVDQ_NVFP4>(p, a, W.Mp, stream)
+                                             : launch_act<SVDQ_INT4_G64>(p, a, W.Mp, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant_kernel launch");
   return launch_status("act_quant_kernel launch");
 }
 

@@ -12,13 +12,15 @@
 //   wq          NVFP4: weight tiles (below), [N/128][K/256] x 20480 bytes
 //               INT4:  N x K bytes, the code as an E4M3 byte (exact for -8..7)
 //   ws          NVFP4: empty (the scales live in the weight tiles)
-//               INT4:  fp32 [K/64][N]
+//               INT4:  fp32 group scales, blocked [K/128][N/256][2][256]
+//               (one 128-wide K slab of a 256-column tile is one contiguous 2 KB)
 //   bias        N fp32
 //
 // Workspace for M tokens:
 //   xq   NVFP4: activation tiles (below), [Mp/128][K/256] x 18432 bytes
 //        INT4:  M x K bytes (code as E4M3 byte)
-//   xs   NVFP4: empty;  INT4: fp32 [K/64][Mp], Mp = ceil(M/128)*128
+//   xs   NVFP4: empty;  INT4: fp32 group scales, blocked [K/128][Mp/128][2][128],
+//        Mp = ceil(M/128)*128 (one K slab of a 128-token tile is one contiguous 1 KB)
 //   ux   M x lrw bf16: [u'_hi | u'_lo (| u'_hi) | 0 pad], u' = u / (s_gX s_gW) (NVFP4) or u (INT4)
 //        (NVFP4: as low-rank tiles over Mp rows; INT4: row-major)
 //
@@ -131,6 +133,15 @@ SVDQ_HD inline size_t sf_offset(int64_t row, int64_t blk, int64_t kblocks) {
   const int64_t atom = (row / 128) * (kblocks / 4) + blk / 4;
   const int64_t r = row % 128;
   return (size_t)(atom * 512 + (r % 32) * 16 + (r / 32) * 4 + (blk % 4));
+}
+
+// Index (in floats) of INT4 group scale g of token m / output feature n in the
+// blocked scale arrays described above.
+SVDQ_HD inline size_t int4_sx_index(int64_t g, int64_t m, int64_t Mp) {
+  return ((size_t)(g >> 1) * (size_t)(Mp / 128) + (size_t)(m / 128)) * 256 + (size_t)(g & 1) * 128 + (size_t)(m % 128);
+}
+SVDQ_HD inline size_t int4_sw_index(int64_t g, int64_t n, int64_t N) {
+  return ((size_t)(g >> 1) * (size_t)(N / 256) + (size_t)(n / 256)) * 512 + (size_t)(g & 1) * 256 + (size_t)(n % 256);
 }
 
 // Byte offset of (row r, byte c) inside a 128 x 128-byte tile with the 128-byte swizzle.

@@ -225,7 +225,7 @@ __device__ __forceinline__ void quantize16(const float (&xh)[16], int64_t m, int
     if (m < a.M)
       *reinterpret_cast<uint4*>(a.xq + (size_t)m * K + kk) =
           make_uint4(w[0] | (w[1] << 16), w[2] | (w[3] << 16), w[4] | (w[5] << 16), w[6] | (w[7] << 16));
-    if (((threadIdx.x & 3) == 0) && m < a.Mp) reinterpret_cast<float*>(a.xs)[(size_t)(kk / 64) * a.Mp + m] = s;
+    if (((threadIdx.x & 3) == 0) && m < a.Mp) reinterpret_cast<float*>(a.xs)[int4_sx_index(kk / 64, m, a.Mp)] = s;
   }
 }
 
@@ -733,19 +733,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
 // INT4 codes live as E4M3 bytes (exact for -8..7), so each group of 64 is two
 // kind::f8f6f4 MMAs whose fp32 partial sum is an exact integer.  The per-group
 // scales sx[m,g] sw[n,g] cannot enter the MMA, so every group's partial is
-// drained from TMEM and folded on the CUDA cores:  acc += P_g * sx * sw.
-// TMEM: two 256-column partial buffers (MMA writes one while the epilogue
-// folds the other).  The low-rank product u L2 is sequence step 0 (scale 1).
-// Warps: 0 TMA producer, 1 MMA issuer, 2-9 fold/epilogue (lane quarter
-// warp % 4, column half (warp - 2) / 4).
+// drained from TMEM and folded on the CUDA cores, two columns per instruction
+// (f32x2):  acc += (P_g * sw) * sx.
+// Persistent, one CTA per SM over 128 x 256 output tiles (n fastest).
+// TMEM: two 256-column partial buffers; the MMA issuer fills one while the
+// fold warps drain the other, across tile boundaries.  The low-rank product
+// u L2 is each tile's first partial (scale 1).
+// Shared memory: a 4-deep ring of K slabs (128 bytes = two groups: A 16 KB,
+// B 32 KB, by 2D TMA), a ring of the slabs' group scales (one 1 KB and one
+// 2 KB bulk copy from the blocked scale arrays), and one 2 KB output chunk per
+// fold warp (32 rows x 32 bf16 columns, 64-byte swizzle) for TMA stores.
+// Warps: 0 producer, 1 TMEM owner + MMA issuer, 2-3 idle [72 regs];
+// 4-11 fold / epilogue, lane quarter warp % 4, column half (warp - 4) / 4 [216]
+// (4 x 32 x 72 + 8 x 32 x 216 = the 384 x 168 registers of the launch).
 constexpr int kI4StageBytes = kABytes + kBBytes;   // A/B ring: 2 groups per stage
 constexpr int kI4ScaleSlot = 2 * kBM * 4 + 2 * kBN * 4;  // sx[2][128] + sw[2][256] fp32 = 3072
 constexpr int kI4Epi = 8;
+constexpr int kI4Threads = 12 * 32;
+constexpr int kI4Chunk = 32 * 64;                  // 32 rows x 32 bf16 columns
+constexpr int kI4Smem = kStages * (kI4StageBytes + kI4ScaleSlot) + kI4Epi * kI4Chunk + 1024;
 
-__global__ void __launch_bounds__(320, 1)
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__global__ void __launch_bounds__(kI4Threads, 1)
     gemm_int4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_ua, const __grid_constant__ CUtensorMap tm_ub,
-                     const GemmArgs g) {
+                     const __grid_constant__ CUtensorMap tm_y, const GemmArgs g) {
   extern __shared__ __align__(1024) uint8_t gsmem_raw[];
   __shared__ uint64_t full_bar[kStages], empty_bar[kStages], sfull_bar[kStages], sempty_bar[kStages];
   __shared__ uint64_t pfull_bar[2], pempty_bar[2], drain_bar;
@@ -754,11 +784,11 @@ __global__ void __launch_bounds__(320, 1)
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sring = smem + kStages * kI4StageBytes;   // scale slots
+  uint8_t* ychunks = sring + kStages * kI4ScaleSlot;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nt = blockIdx.x, mt = blockIdx.y;
-  const int n0 = nt * kBN;
-  const int64_t m0 = (int64_t)mt * kBM;
-  const int total = g.lr_iters + g.k_iters;
+  const int n_tiles = g.N / kBN;
+  const int num_tiles = n_tiles * (int)(g.Mp / kBM);
+  const int total = g.lr_iters + g.k_iters;   // ring steps per tile
   const int has_lr = g.lr_iters > 0;
   volatile int* abort_flag = &abort_sh;
 
@@ -773,7 +803,7 @@ __global__ void __launch_bounds__(320, 1)
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tm_a); prefetch_tmap(&tm_b);
+    prefetch_tmap(&tm_a); prefetch_tmap(&tm_b); prefetch_tmap(&tm_y);
     if (has_lr) { prefetch_tmap(&tm_ua); prefetch_tmap(&tm_ub); }
   }
   if (warp == 1) { tmem_alloc(&tmem_base_sh, 512); tmem_relinquish(); }
@@ -782,85 +812,88 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tbase = tmem_base_sh;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      int issued = 0, sissued = 0;
-      for (int it = 0; it < total; ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        if (!mbar_wait(&empty_bar[s], ph ^ 1, abort_flag)) break;
-        uint8_t* st = smem + s * kI4StageBytes;
-        if (it < g.lr_iters) {
+  if (warp < 4) {
+    regs_dec<72>();
+    if (warp == 0 && lane == 0) {
+      int it = 0, issued = 0, sk = 0, sissued = 0;
+      bool dead = false;
+      for (int tile = blockIdx.x; tile < num_tiles && !dead; tile += gridDim.x) {
+        const int mt = tile / n_tiles, nt = tile % n_tiles;
+        const int n0 = nt * kBN;
+        const int64_t m0 = (int64_t)mt * kBM;
+        for (int j = 0; j < total; ++j, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait(&empty_bar[s], ((it / kStages) & 1) ^ 1, abort_flag)) { dead = true; break; }
+          uint8_t* st = smem + s * kI4StageBytes;
           mbar_arrive_expect_tx(&full_bar[s], kABytes + kBBytes);
-          tma_load_2d(st, &tm_ua, &full_bar[s], it * 64, (int)m0);
-          tma_load_2d(st + kABytes, &tm_ub, &full_bar[s], it * 64, n0);
-        } else {
-          const int kt = it - g.lr_iters;
-          mbar_arrive_expect_tx(&full_bar[s], kABytes + kBBytes);
-          tma_load_2d(st, &tm_a, &full_bar[s], kt * 128, (int)m0);
-          tma_load_2d(st + kABytes, &tm_b, &full_bar[s], kt * 128, n0);
-          // group scales of this slab go to the scale ring (read by the fold warps)
-          const int ss = kt % kStages;
-          if (!mbar_wait(&sempty_bar[ss], ((kt / kStages) & 1) ^ 1, abort_flag)) { issued = it + 1; break; }
-          uint8_t* slot = sring + ss * kI4ScaleSlot;
-          const float* sx = reinterpret_cast<const float*>(g.sfa);
-          const float* sw = reinterpret_cast<const float*>(g.sfb);
-          mbar_arrive_expect_tx(&sfull_bar[ss], kI4ScaleSlot);
-          for (int h = 0; h < 2; ++h) {
-            const int grp = 2 * kt + h;
-            bulk_load(slot + h * kBM * 4, sx + (size_t)grp * g.Mp + m0, kBM * 4, &sfull_bar[ss]);
-            bulk_load(slot + 2 * kBM * 4 + h * kBN * 4, sw + (size_t)grp * g.N + n0, kBN * 4, &sfull_bar[ss]);
+          if (j < g.lr_iters) {
+            tma_load_2d(st, &tm_ua, &full_bar[s], j * 64, (int)m0);
+            tma_load_2d(st + kABytes, &tm_ub, &full_bar[s], j * 64, n0);
+          } else {
+            const int kt = j - g.lr_iters;
+            tma_load_2d(st, &tm_a, &full_bar[s], kt * 128, (int)m0);
+            tma_load_2d(st + kABytes, &tm_b, &full_bar[s], kt * 128, n0);
+            // the slab's two groups of scales (blocked layouts: one copy each)
+            const int ss = sk % kStages;
+            if (!mbar_wait(&sempty_bar[ss], ((sk / kStages) & 1) ^ 1, abort_flag)) { issued = it + 1; dead = true; break; }
+            uint8_t* slot = sring + ss * kI4ScaleSlot;
+            const float* sx = reinterpret_cast<const float*>(g.sfa) + ((size_t)kt * (size_t)(g.Mp / kBM) + mt) * 256;
+            const float* sw = reinterpret_cast<const float*>(g.sfb) + ((size_t)kt * n_tiles + nt) * 512;
+            mbar_arrive_expect_tx(&sfull_bar[ss], kI4ScaleSlot);
+            bulk_load(slot, sx, 2 * kBM * 4, &sfull_bar[ss]);
+            bulk_load(slot + 2 * kBM * 4, sw, 2 * kBN * 4, &sfull_bar[ss]);
+            ++sk;
+            sissued = sk;
           }
-          sissued = kt + 1;
+          issued = it + 1;
         }
-        issued = it + 1;
       }
       if (*abort_flag) {
-        for (int it = issued - 1; it >= 0 && it >= issued - kStages; --it)
-          mbar_drain(&full_bar[it % kStages], (it / kStages) & 1);
-        for (int kt = sissued - 1; kt >= 0 && kt >= sissued - kStages; --kt)
-          mbar_drain(&sfull_bar[kt % kStages], (kt / kStages) & 1);
+        for (int i = issued - 1; i >= 0 && i >= issued - kStages; --i)
+          mbar_drain(&full_bar[i % kStages], (i / kStages) & 1);
+        for (int i = sissued - 1; i >= 0 && i >= sissued - kStages; --i)
+          mbar_drain(&sfull_bar[i % kStages], (i / kStages) & 1);
       }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
       const uint32_t id_lr = idesc_f16_bf16(kBM, kBN);
       const uint32_t id_f8 = idesc_f8_e4m3(kBM, kBN);
-      int seq = 0;     // partial-buffer sequence: LR product (if any), then groups
+      int it = 0, seq = 0;   // seq: partial-buffer sequence over all tiles
       bool dead = false;
-      for (int it = 0; it < total && !dead; ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        if (!mbar_wait(&full_bar[s], ph, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + s * kI4StageBytes);
-        const uint32_t b_addr = a_addr + kABytes;
-        if (it < g.lr_iters) {
-          if (it == 0) {
-            if (!mbar_wait(&pempty_bar[0], 1, abort_flag)) break;
-            tc_fence_after();
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            mma_f16(tbase, desc_k_sw128(a_addr + 32 * j), desc_k_sw128(b_addr + 32 * j), id_lr,
-                    (it | j) != 0);
-          if (it == g.lr_iters - 1) { mma_commit(&pfull_bar[0]); seq = 1; }
-        } else {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
+      for (int tile = blockIdx.x; tile < num_tiles && !dead; tile += gridDim.x) {
+        for (int j = 0; j < total && !dead; ++j, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait(&full_bar[s], (it / kStages) & 1, abort_flag)) { dead = true; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * kI4StageBytes);
+          const uint32_t b_addr = a_addr + kABytes;
+          if (j < g.lr_iters) {
             const int buf = seq & 1;
-            if (!mbar_wait(&pempty_bar[buf], ((seq >> 1) & 1) ^ 1, abort_flag)) { dead = true; break; }
-            tc_fence_after();
-            const uint32_t d = tbase + 256 * buf;
+            if (j == 0) {
+              if (!mbar_wait(&pempty_bar[buf], ((seq >> 1) & 1) ^ 1, abort_flag)) { dead = true; break; }
+              tc_fence_after();
+            }
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
-              mma_f8(d, desc_k_sw128(a_addr + 64 * h + 32 * j), desc_k_sw128(b_addr + 64 * h + 32 * j), id_f8,
-                     j != 0);
-            mma_commit(&pfull_bar[buf]);
-            ++seq;
+            for (int q = 0; q < 4; ++q)
+              mma_f16(tbase + 256 * buf, desc_k_sw128(a_addr + 32 * q), desc_k_sw128(b_addr + 32 * q), id_lr,
+                      (j | q) != 0);
+            if (j == g.lr_iters - 1) { mma_commit(&pfull_bar[buf]); ++seq; }
+          } else {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int buf = seq & 1;
+              if (!mbar_wait(&pempty_bar[buf], ((seq >> 1) & 1) ^ 1, abort_flag)) { dead = true; break; }
+              tc_fence_after();
+              const uint32_t d = tbase + 256 * buf;
+#pragma unroll
+              for (int q = 0; q < 2; ++q)
+                mma_f8(d, desc_k_sw128(a_addr + 64 * h + 32 * q), desc_k_sw128(b_addr + 64 * h + 32 * q), id_f8,
+                       q != 0);
+              mma_commit(&pfull_bar[buf]);
+              ++seq;
+            }
           }
+          mma_commit(&empty_bar[s]);
         }
-        mma_commit(&empty_bar[s]);
       }
       if (*abort_flag) {
         // wait for this thread's MMAs before TMEM is released
@@ -869,75 +902,114 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
   } else {
-    // fold / epilogue warps 2..9
-    const int e = warp - 2;
+    regs_inc<216>();
+    // fold / epilogue warps 4..11
+    const int e = warp - 4;
     const int q = warp & 3;                 // TMEM lane quarter
     const int ch = e >> 2;                  // column half
-    const int64_t m = m0 + q * 32 + lane;
     const int row_in_tile = q * 32 + lane;
-    float acc[128];
-#pragma unroll
-    for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
-    int seq = 0;
-    bool ok = true;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
-    if (has_lr) {
-      ok = mbar_wait(&pfull_bar[0], 0, abort_flag);
-      tc_fence_after();
-      if (ok) {
+    uint8_t* ybuf = ychunks + e * kI4Chunk;
+    int seq = 0, sk = 0;
+    bool ok = true;
+    uint64_t acc[64];   // 128 columns as f32 pairs
+    // drain partial buffer `buf` into acc: acc += (P * sw) * sx, 64 columns at a time;
+    // the buffer is released once both halves are in registers
+    auto fold = [&](int buf, const float* swp, float sxm, bool plain) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld_32cols(tbase + lane_addr + ch * 128 + c * 32, v);
-          tmem_ld_wait();
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t v[64];
+        tmem_ld_32cols(tbase + lane_addr + 256 * buf + ch * 128 + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
+        tmem_ld_32cols(tbase + lane_addr + 256 * buf + ch * 128 + hh * 64 + 32,
+                       *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        tmem_ld_wait();
+        if (hh == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&pempty_bar[buf]);
+        }
+        if (plain) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) acc[c * 32 + j] = __uint_as_float(v[j]);
+          for (int j = 0; j < 32; ++j) acc[hh * 32 + j] = f2_pack(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+        } else {
+          const uint64_t sx2 = f2_pack(sxm, sxm);
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float4 w4 = *reinterpret_cast<const float4*>(swp + hh * 64 + 2 * j);
+            const uint64_t p0 = f2_mul(f2_pack(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])),
+                                       f2_pack(w4.x, w4.y));
+            const uint64_t p1 = f2_mul(f2_pack(__uint_as_float(v[2 * j + 2]), __uint_as_float(v[2 * j + 3])),
+                                       f2_pack(w4.z, w4.w));
+            acc[hh * 32 + j] = f2_fma(p0, sx2, acc[hh * 32 + j]);
+            acc[hh * 32 + j + 1] = f2_fma(p1, sx2, acc[hh * 32 + j + 1]);
+          }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&pempty_bar[0]);
-      seq = 1;
-    }
-    for (int kt = 0; kt < g.k_iters && ok; ++kt) {
-      const int ss = kt % kStages;
-      if (!mbar_wait(&sfull_bar[ss], (kt / kStages) & 1, abort_flag)) { ok = false; break; }
-      const float* slot = reinterpret_cast<const float*>(sring + ss * kI4ScaleSlot);
-      for (int h = 0; h < 2; ++h) {
+    };
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const int mt = tile / n_tiles, nt = tile % n_tiles;
+      const int col0 = nt * kBN + ch * 128;
+      const int64_t m0 = (int64_t)mt * kBM;
+      if (has_lr) {
         const int buf = seq & 1;
         if (!mbar_wait(&pfull_bar[buf], (seq >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const float sxm = slot[h * kBM + row_in_tile];
-        const float* swp = slot + 2 * kBM + h * kBN + ch * 128;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld_32cols(tbase + lane_addr + 256 * buf + ch * 128 + c * 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            acc[c * 32 + j] = fmaf(__uint_as_float(v[j]), sxm * swp[c * 32 + j], acc[c * 32 + j]);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&pempty_bar[buf]);
+        fold(buf, nullptr, 1.0f, true);
         ++seq;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) acc[j] = 0ull;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sempty_bar[ss]);
-    }
-    if (ok && m < g.M) {
+      for (int kt = 0; kt < g.k_iters && ok; ++kt, ++sk) {
+        const int ss = sk % kStages;
+        if (!mbar_wait(&sfull_bar[ss], (sk / kStages) & 1, abort_flag)) { ok = false; break; }
+        const float* slot = reinterpret_cast<const float*>(sring + ss * kI4ScaleSlot);
+        for (int h = 0; h < 2; ++h) {
+          const int buf = seq & 1;
+          if (!mbar_wait(&pfull_bar[buf], (seq >> 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          fold(buf, slot + 2 * kBM + h * kBN + ch * 128, slot[h * kBM + row_in_tile], false);
+          ++seq;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sempty_bar[ss]);
+      }
+      if (!ok) break;
+      // epilogue: y = acc + bias -> bf16, 32-column chunks through shared memory
+      const int64_t row0 = m0 + q * 32;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        float bias[32];
+        const float bl = __ldg(g.bias + col0 + 32 * c + lane);   // bias of column 32c + lane
+        uint4 pk[4];
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-          const float4 b4 = __ldg(reinterpret_cast<const float4*>(g.bias + n0 + ch * 128 + c * 32 + j));
-          bias[j] = b4.x; bias[j + 1] = b4.y; bias[j + 2] = b4.z; bias[j + 3] = b4.w;
+        for (int t = 0; t < 4; ++t) {
+          uint32_t w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int jj = 16 * c + 4 * t + i;   // f32 pair index: columns 2jj, 2jj+1
+            float y0, y1;
+            f2_unpack(acc[jj], y0, y1);
+            y0 += __shfl_sync(0xffffffffu, bl, (2 * jj) & 31);
+            y1 += __shfl_sync(0xffffffffu, bl, (2 * jj + 1) & 31);
+            w[i] = (uint32_t)bf16_rn(y0) | ((uint32_t)bf16_rn(y1) << 16);
+          }
+          pk[t] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        store_row32(g.Y + (size_t)m * g.N + n0 + ch * 128 + c * 32, acc + c * 32, bias, 1.0f);
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          *reinterpret_cast<uint4*>(ybuf + lane * 64 + ((t ^ ((lane >> 1) & 3)) << 4)) = pk[t];
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < g.M) {
+          tma_store_2d(&tm_y, ybuf, col0 + 32 * c, (int)row0);
+          bulk_commit();
+        }
       }
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -1168,7 +1240,7 @@ svdq_status device_ready() {
     d.ok = prop.major == 10 && prop.minor == 0;
     d.sms = prop.multiProcessorCount;
     if (d.ok) {
-      const int i4_smem = dev::kStages * (dev::kI4StageBytes + dev::kI4ScaleSlot) + 1024;
+      const int i4_smem = dev::kI4Smem;
       d.ok = cudaFuncSetAttribute(dev::gemm_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   dev::kP_Smem) == cudaSuccess &&
              cudaFuncSetAttribute(dev::gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1301,10 +1373,12 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
     dev::gemm_nvfp4_pair_kernel<<<2 * pairs, dev::kP_Threads, dev::kP_Smem, stream>>>(g, tm_y);
     return launch_status("gemm_nvfp4_pair_kernel launch");
   }
-  CUtensorMap tm_a, tm_b, tm_ua, tm_ub;
+  CUtensorMap tm_a, tm_b, tm_ua, tm_ub, tm_y;
   const uint64_t krow = (uint64_t)K;
   bool ok = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + W.off_xq, krow, (uint64_t)M, krow, 128, dev::kBM) &&
-            make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, blob + B.off_wq, krow, (uint64_t)N, krow, 128, dev::kBN);
+            make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, blob + B.off_wq, krow, (uint64_t)N, krow, 128, dev::kBN) &&
+            make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 32, 32,
+                     CU_TENSOR_MAP_SWIZZLE_64B);
   if (r > 0) {
     ok = ok && make_map(&tm_ua, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + W.off_ux, (uint64_t)lrw, (uint64_t)M,
                         (uint64_t)lrw * 2, 64, dev::kBM) &&
@@ -1324,9 +1398,9 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
   g.hdr = reinterpret_cast<const BlobHeader*>(blob);
   g.Y = static_cast<uint16_t*>(Y);
   g.Mp = W.Mp;
-  const dim3 grid((unsigned)(N / dev::kBN), (unsigned)(W.Mp / dev::kBM));
-  dev::gemm_int4_kernel<<<grid, 320, dev::kStages * (dev::kI4StageBytes + dev::kI4ScaleSlot) + 1024, stream>>>(
-      tm_a, tm_b, tm_ua, tm_ub, g);
+  const int tiles = (N / dev::kBN) * (int)(W.Mp / dev::kBM);
+  const int grid = std::max(1, std::min(tiles, num_sms()));
+  dev::gemm_int4_kernel<<<grid, dev::kI4Threads, dev::kI4Smem, stream>>>(tm_a, tm_b, tm_ua, tm_ub, tm_y, g);
   return launch_status("gemm kernel launch");
 }
 

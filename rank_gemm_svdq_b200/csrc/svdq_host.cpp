@@ -445,14 +445,14 @@ svdq_status svdq_prepare(const svdq_params* p, const float* Wt, const float* bia
   BlobHeader* h = (BlobHeader*)base;
   h->s_gw = 1.0f;
   if (p->fmt == SVDQ_INT4_G64) {
-    float* sw = (float*)wsb;                                   // [K/64][N]
+    float* sw = (float*)wsb;                                   // blocked, int4_sw_index
 #pragma omp parallel for schedule(static)
     for (int n = 0; n < N; ++n) {
       std::vector<int8_t> q(K);
       std::vector<float> s(K / kGroupInt4);
       int4_quant_row(&R[(size_t)n * K], K, q.data(), s.data());
       for (int j = 0; j < K; ++j) wq[(size_t)n * K + j] = e4m3_encode((float)q[j]);
-      for (int g = 0; g < K / kGroupInt4; ++g) sw[(size_t)g * N + n] = s[g];
+      for (int g = 0; g < K / kGroupInt4; ++g) sw[int4_sw_index(g, n, N)] = s[g];
     }
   } else {
     float amax = 0.0f;
@@ -602,7 +602,7 @@ svdq_status svdq_blob_export(const svdq_params* p, const void* blob, float* inv_
       const float* sw = (const float*)wsb;
       const int G = K / kGroupInt4;
       for (int n = 0; n < N; ++n)
-        for (int g = 0; g < G; ++g) o[(size_t)n * G + g] = sw[(size_t)g * N + n];
+        for (int g = 0; g < G; ++g) o[(size_t)n * G + g] = sw[int4_sw_index(g, n, N)];
     }
   }
   if (tscales) { tscales[0] = h->s_gx; tscales[1] = h->s_gw; }
@@ -643,7 +643,7 @@ svdq_status svdq_decode_act_host(const svdq_params* p, const uint8_t* ws, int64_
       const float* sx = (const float*)(ws + W.off_xs);
       const int G = K / kGroupInt4;
       for (int64_t m = 0; m < M; ++m)
-        for (int g = 0; g < G; ++g) o[(size_t)m * G + g] = sx[(size_t)g * W.Mp + m];
+        for (int g = 0; g < G; ++g) o[(size_t)m * G + g] = sx[int4_sx_index(g, m, W.Mp)];
     }
   }
   if (u) {

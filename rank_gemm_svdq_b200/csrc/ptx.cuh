@@ -100,6 +100,18 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// Prefetch `bytes` (multiple of 16, 16-byte aligned) of global memory into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start before the previous kernel of the stream ends;
+// griddep_wait blocks the calling thread until that kernel has completed and
+// its memory is visible.  griddep_launch lets the next kernel start early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // 2-CTA TMA load (cta_group::2): writes this CTA's shared memory and signals
 // the mbarrier at `bar_cluster` (a shared::cluster address, here always the
 // pair leader's barrier).  No multicast.

@@ -249,6 +249,7 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
   auto xs16 = [&](int b) { return xs16_base + b * kActRows * kActStride; };
   auto l1sb = [&](int b) { return l1s_base + b * r * kActStride; };
 
+  griddep_launch();   // the GEMM may start its prologue on idle SMs
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int KS = a.ks;
   const int kidx = KS > 1 ? (int)cluster_ctarank() : 0;
@@ -557,6 +558,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
   if (warp == 0) {
     regs_dec<56>();
     if (lane == 0) {
+      // The weights do not depend on the activation kernel: when every pair
+      // has a single tile (few tokens), pull this CTA's weight tiles into L2
+      // while that kernel runs; then wait for it before touching the workspace.
+      if (num_tiles <= pairs && pair < num_tiles) {   // one tile per pair: weight streaming dominates
+        const size_t nb0 = (size_t)(2 * (pair % n_tiles) + (int)rank);
+        for (int kt = 0; kt < ksl; ++kt) bulk_prefetch_l2(g.wtiles + (nb0 * ksl + kt) * kWTile, kWTile);
+      }
+      griddep_wait();
       int it = 0, issued = 0;
       bool dead = false;
       for (int tile = pair; tile < num_tiles && !dead; tile += pairs) {
@@ -815,6 +824,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   if (warp < 4) {
     regs_dec<72>();
     if (warp == 0 && lane == 0) {
+      griddep_wait();   // the workspace comes from the activation kernel
       int it = 0, issued = 0, sk = 0, sissued = 0;
       bool dead = false;
       for (int tile = blockIdx.x; tile < num_tiles && !dead; tile += gridDim.x) {
@@ -1370,7 +1380,18 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
       return cuda_fail(cudaErrorInvalidValue, "tensor map encode (Y)");
     const int tiles = (N / 256) * (int)(W.Mp / 256);
     const int pairs = std::max(1, std::min(tiles, num_sms() / 2));
-    dev::gemm_nvfp4_pair_kernel<<<2 * pairs, dev::kP_Threads, dev::kP_Smem, stream>>>(g, tm_y);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(dev::kP_Threads);
+    cfg.dynamicSmemBytes = dev::kP_Smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_pair_kernel, g, tm_y);
+    if (e != cudaSuccess) return cuda_fail(e, "gemm_nvfp4_pair_kernel launch");
     return launch_status("gemm_nvfp4_pair_kernel launch");
   }
   CUtensorMap tm_a, tm_b, tm_ua, tm_ub, tm_y;
@@ -1400,7 +1421,18 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
   g.Mp = W.Mp;
   const int tiles = (N / dev::kBN) * (int)(W.Mp / dev::kBM);
   const int grid = std::max(1, std::min(tiles, num_sms()));
-  dev::gemm_int4_kernel<<<grid, dev::kI4Threads, dev::kI4Smem, stream>>>(tm_a, tm_b, tm_ua, tm_ub, tm_y, g);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(dev::kI4Threads);
+  cfg.dynamicSmemBytes = dev::kI4Smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, dev::gemm_int4_kernel, tm_a, tm_b, tm_ua, tm_ub, tm_y, g);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm_int4_kernel launch");
   return launch_status("gemm kernel launch");
 }
 

@@ -122,7 +122,12 @@ __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_
 SVDQ_HD inline int act_l1_bufs(int r) {
   return (2 * kActRows + 3 * r) * kActStride * 2 <= kActSmemMax ? 3 : 2;
 }
-SVDQ_HD inline int act_smem_bytes(int r) { return (2 * kActRows + act_l1_bufs(r) * r) * kActStride * 2; }
+SVDQ_HD inline int act_ring_bytes(int r) { return (2 * kActRows + act_l1_bufs(r) * r) * kActStride * 2; }
+// The CTA's slice of inv_lambda (k_range floats) also sits in shared memory when it fits.
+SVDQ_HD inline bool act_il_in_smem(int r, int k_range) { return act_ring_bytes(r) + k_range * 4 <= kActSmemMax; }
+SVDQ_HD inline int act_smem_bytes(int r, int k_range) {
+  return act_ring_bytes(r) + (act_il_in_smem(r, k_range) ? k_range * 4 : 0);
+}
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& a0, uint32_t& a1, uint32_t& a2,
                                             uint32_t& a3) {
@@ -300,6 +305,23 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
   };
   for (int c = 0; c < lead; ++c) stage_l1(c);
 
+  // inv_lambda of this CTA's K range, read by every token.  In shared memory
+  // (when it fits) each 256-wide chunk is stored as [q][l][4] -- element
+  // 16 l + 4 q + j at (16 q + l) * 4 + j -- so that lane l's four float4
+  // reads of its 16 elements hit distinct banks.
+  const int k_range = cpk * kActChunk;
+  const bool il_smem = act_il_in_smem(r, k_range);
+  const float* il_s = reinterpret_cast<const float*>(act_smem + act_ring_bytes(r) / 2);
+  if (il_smem) {
+    float* dst = reinterpret_cast<float*>(act_smem + act_ring_bytes(r) / 2);
+    const float4* src = reinterpret_cast<const float4*>(a.inv_lambda + (size_t)c0 * kActChunk);
+    for (int i = tid; i < k_range / 4; i += kActThreads) {
+      const int ch = i / 64, w = i % 64, l = w >> 2, q = w & 3;   // float4 w of chunk ch = lane l, quarter q
+      reinterpret_cast<float4*>(dst + ch * kActChunk)[q * 16 + l] = __ldg(src + i);
+    }
+    __syncthreads();
+  }
+
   for (int c = 0; c < cpk; ++c) {
     const int k0 = (c0 + c) * kActChunk;
     const int buf = c & 1;
@@ -308,7 +330,8 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
     float il[16];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float4 f = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + kk + 4 * i));
+      const float4 f = il_smem ? reinterpret_cast<const float4*>(il_s + c * kActChunk)[i * 16 + (lane & 15)]
+                               : __ldg(reinterpret_cast<const float4*>(a.inv_lambda + kk + 4 * i));
       il[4 * i] = f.x; il[4 * i + 1] = f.y; il[4 * i + 2] = f.z; il[4 * i + 3] = f.w;
     }
     const uint16_t* x16 = reinterpret_cast<const uint16_t*>(xc);
@@ -1306,7 +1329,7 @@ cudaError_t launch_act(const svdq_params* p, dev::ActArgs a, int64_t Mp, cudaStr
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(Mp / dev::kActRows * a.ks));
   cfg.blockDim = dim3(dev::kActThreads);
-  cfg.dynamicSmemBytes = (size_t)dev::act_smem_bytes(p->rank);
+  cfg.dynamicSmemBytes = (size_t)dev::act_smem_bytes(p->rank, p->K / a.ks);
   cfg.stream = stream;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;

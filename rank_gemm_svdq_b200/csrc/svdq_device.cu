@@ -90,7 +90,7 @@ struct ActArgs {
 
 constexpr int kActRows = 32;     // tokens per CTA
 constexpr int kActThreads = 512;
-constexpr int kActSmemMax = 232448;
+constexpr int kActSmemMax = 232448 - 4096;   // dynamic; the kernel also has 2 KB of static tables
 constexpr int kActChunk = 256;   // K elements per step
 constexpr int kActStride = kActChunk + 8;  // padded smem row (bf16/fp16 elements)
 
@@ -173,8 +173,11 @@ __device__ __forceinline__ uint32_t pack_half2_rn(float lo, float hi) {
 // block, or a quarter of an INT4 group of 64 spread over 4 lanes) and store
 // codes / scales.
 template <int FMT>
+// dq: NVFP4 per-code tables in shared memory, dq[e] = E4M3(e) * s_gX and
+// dq[256 + e] = its round-to-nearest reciprocal (0 where the FMA-corrected
+// division is not valid); unused for INT4.
 __device__ __forceinline__ void quantize16(const float (&xh)[16], int64_t m, int kk, const ActArgs& a,
-                                           float s_gx, float six_sg, float r6) {
+                                           float s_gx, float six_sg, float r6, const float* dq) {
   const int K = a.K;
   float amax = 0.0f;
 #pragma unroll
@@ -182,11 +185,11 @@ __device__ __forceinline__ void quantize16(const float (&xh)[16], int64_t m, int
   if constexpr (FMT == SVDQ_NVFP4) {
     const float ratio = r6 != 0.0f ? div_by_recip(amax, six_sg, r6) : __fdiv_rn(amax, six_sg);
     const uint32_t e = cvt_e4m3x2(0.0f, ratio) & 0xFFu;
-    const float d = __fmul_rn(e4m3_val(e), s_gx);
+    const float d = dq[e];
+    const float rd = dq[256 + e];
     uint32_t p0 = 0, p1 = 0;
     if (d != 0.0f) {
-      if (recip_ok(d)) {
-        const float rd = __frcp_rn(d);
+      if (rd != 0.0f) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           p0 |= cvt_e2m1x2(div_by_recip(xh[2 * i + 1], d, rd), div_by_recip(xh[2 * i], d, rd)) << (8 * i);
@@ -311,6 +314,14 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
   // reads of its 16 elements hit distinct banks.
   const int k_range = cpk * kActChunk;
   const bool il_smem = act_il_in_smem(r, k_range);
+  // NVFP4 per-code block-scale tables (see quantize16): same values as
+  // computing them per block, looked up instead
+  __shared__ float dq_tab[512];
+  if (FMT == SVDQ_NVFP4 && tid < 256) {
+    const float d = __fmul_rn(e4m3_val((uint32_t)tid), s_gx);
+    dq_tab[tid] = d;
+    dq_tab[256 + tid] = (d != 0.0f && recip_ok(d)) ? __frcp_rn(d) : 0.0f;
+  }
   const float* il_s = reinterpret_cast<const float*>(act_smem + act_ring_bytes(r) / 2);
   if (il_smem) {
     float* dst = reinterpret_cast<float*>(act_smem + act_ring_bytes(r) / 2);
@@ -319,8 +330,8 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
       const int ch = i / 64, w = i % 64, l = w >> 2, q = w & 3;   // float4 w of chunk ch = lane l, quarter q
       reinterpret_cast<float4*>(dst + ch * kActChunk)[q * 16 + l] = __ldg(src + i);
     }
-    __syncthreads();
   }
+  __syncthreads();
 
   for (int c = 0; c < cpk; ++c) {
     const int k0 = (c0 + c) * kActChunk;
@@ -338,7 +349,7 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
     float xh[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) xh[i] = __fmul_rn(half_to_f32<DT>(x16[i]), il[i]);
-    quantize16<FMT>(xh, m, kk, a, s_gx, six_sg, r6);
+    quantize16<FMT>(xh, m, kk, a, s_gx, six_sg, r6, dq_tab);
     uint4 o0, o1;
     o0.x = pack_half2_rn<DT>(xh[0], xh[1]);   o0.y = pack_half2_rn<DT>(xh[2], xh[3]);
     o0.z = pack_half2_rn<DT>(xh[4], xh[5]);   o0.w = pack_half2_rn<DT>(xh[6], xh[7]);

@@ -23,6 +23,7 @@
 //        Mp = ceil(M/128)*128 (one K slab of a 128-token tile is one contiguous 1 KB)
 //   ux   M x lrw bf16: [u'_hi | u'_lo (| u'_hi) | 0 pad], u' = u / (s_gX s_gW) (NVFP4) or u (INT4)
 //        (NVFP4: as low-rank tiles over Mp rows; INT4: row-major)
+//   part, cnt   NVFP4 K-split scratch when nvfp4_split_k_eligible (below), else empty
 //
 // NVFP4 operand tiles (what one bulk copy brings into shared memory, ready
 // for the tensor core): 128 rows x one K slab of 256 elements.  The E2M1
@@ -105,9 +106,18 @@ inline BlobLayout blob_layout(const svdq_params& p) {
 }
 
 struct WsLayout {
-  size_t off_xq, off_xs, off_ux, total;
+  size_t off_xq, off_xs, off_ux, off_part, off_cnt, total;
   int64_t Mp;  // M rounded up to the GEMM's row tile (256 NVFP4, 128 INT4)
 };
+
+// NVFP4 with few tokens and few output tiles: the GEMM may split K over up to
+// kMaxKSplit CTA pairs per tile; the workspace then also holds the fp32
+// partial sums [ks][M][N] and one arrival counter per tile region [tiles][16]
+// (zeroed by the activation kernel of the same call).
+constexpr int kMaxKSplit = 8;
+inline bool nvfp4_split_k_eligible(const svdq_params& p, int64_t M) {
+  return p.fmt == SVDQ_NVFP4 && M >= 1 && M <= 64 && p.N / 256 <= 37;
+}
 
 inline WsLayout ws_layout(const svdq_params& p, int64_t M) {
   WsLayout L{};
@@ -123,6 +133,12 @@ inline WsLayout ws_layout(const svdq_params& p, int64_t M) {
   off = align_up(off + (p.fmt == SVDQ_NVFP4 ? 0 : (K / kGroupInt4) * Mp * 4));
   L.off_ux = off;
   off = align_up(off + (p.fmt == SVDQ_NVFP4 ? Mp : (size_t)M) * (size_t)lr_width(p) * 2);
+  L.off_part = L.off_cnt = off;
+  if (nvfp4_split_k_eligible(p, M)) {
+    off = align_up(off + (size_t)kMaxKSplit * (size_t)M * (size_t)p.N * 4);
+    L.off_cnt = off;
+    off = align_up(off + (size_t)(p.N / 256) * (Mp / 256) * 16 * 4);
+  }
   L.total = off > 0 ? off : kAlign;
   return L;
 }

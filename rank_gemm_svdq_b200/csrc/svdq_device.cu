@@ -86,6 +86,8 @@ struct ActArgs {
   uint8_t* xs;
   uint16_t* ux;
   int ks;   // K split: a cluster of ks CTAs shares one group of 32 tokens
+  int* gemm_cnt;   // GEMM K-split arrival counters to clear (or null)
+  int n_cnt;
 };
 
 constexpr int kActRows = 32;     // tokens per CTA
@@ -259,6 +261,8 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
 
   griddep_launch();   // the GEMM may start its prologue on idle SMs
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (blockIdx.x == 0 && a.gemm_cnt)
+    for (int i = tid; i < a.n_cnt; i += kActThreads) a.gemm_cnt[i] = 0;
   const int KS = a.ks;
   const int kidx = KS > 1 ? (int)cluster_ctarank() : 0;
   const int64_t m0 = (int64_t)(blockIdx.x / KS) * kActRows;
@@ -551,6 +555,9 @@ struct PairArgs {
   const float* bias;
   const BlobHeader* hdr;
   uint16_t* Y;
+  int ks;                  // K split (few output tiles): items = tiles x ks
+  float* part;             // ks > 1: fp32 partial sums [ks][M][N]
+  int* cnt;                // ks > 1: arrival counters [tiles][16] (zero between calls)
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
@@ -568,8 +575,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
   const int pair = blockIdx.x >> 1, pairs = gridDim.x >> 1;
   const int n_tiles = g.N / 256;
   const int num_tiles = n_tiles * (int)(g.Mp / 256);
-  const int per_tile = g.lr_iters + g.k_iters;
   const int ksl = g.K / 256;
+  // Work items: output tile x K range.  With g.ks > 1 item (t, kq) covers
+  // slabs [kq cpk, (kq + 1) cpk); only kq = 0 adds the low-rank steps.
+  const int num_items = num_tiles * g.ks;
+  const int cpk = g.k_iters / g.ks;
+  auto item_lr = [&](int item) { return (item % g.ks) == 0 ? g.lr_iters : 0; };
   volatile int* abort_flag = &abort_sh;
 
   if (threadIdx.x == 0) {
@@ -595,26 +606,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
       // The weights do not depend on the activation kernel: when every pair
       // has a single tile (few tokens), pull this CTA's weight tiles into L2
       // while that kernel runs; then wait for it before touching the workspace.
-      if (num_tiles <= pairs && pair < num_tiles) {   // one tile per pair: weight streaming dominates
-        const size_t nb0 = (size_t)(2 * (pair % n_tiles) + (int)rank);
-        for (int kt = 0; kt < ksl; ++kt) bulk_prefetch_l2(g.wtiles + (nb0 * ksl + kt) * kWTile, kWTile);
+      if (num_items <= pairs && pair < num_items) {   // one item per pair: weight streaming dominates
+        const int t0 = pair / g.ks, kq0 = pair % g.ks;
+        const size_t nb0 = (size_t)(2 * (t0 % n_tiles) + (int)rank);
+        for (int kt = kq0 * cpk; kt < (kq0 + 1) * cpk; ++kt)
+          bulk_prefetch_l2(g.wtiles + (nb0 * ksl + kt) * kWTile, kWTile);
       }
       griddep_wait();
       int it = 0, issued = 0;
       bool dead = false;
-      for (int tile = pair; tile < num_tiles && !dead; tile += pairs) {
+      for (int item = pair; item < num_items && !dead; item += pairs) {
+        const int tile = item / g.ks, kq = item % g.ks, lr = item_lr(item);
         const int mt = tile / n_tiles, nt = tile % n_tiles;
         const size_t mb = (size_t)(2 * mt + (int)rank), nb = (size_t)(2 * nt + (int)rank);
-        for (int j = 0; j < per_tile; ++j, ++it) {
+        for (int j = 0; j < lr + cpk; ++j, ++it) {
           const int s = it % kP_Stages;
           if (!mbar_wait(&empty_bar[s], ((it / kP_Stages) & 1) ^ 1, abort_flag)) { give_up_both(); dead = true; break; }
           uint8_t* st = smem + s * kS_Size;
-          if (j < g.lr_iters) {
+          if (j < lr) {
             mbar_arrive_expect_tx(&landed_bar[s], 2 * kLRTile);
             bulk_load(st, g.utiles + (mb * g.lr_iters + j) * kLRTile, kLRTile, &landed_bar[s]);
             bulk_load(st + kS_B, g.l2tiles + (nb * g.lr_iters + j) * kLRTile, kLRTile, &landed_bar[s]);
           } else {
-            const int kt = j - g.lr_iters;
+            const int kt = kq * cpk + (j - lr);
             mbar_arrive_expect_tx(&landed_bar[s], kS_Size);
             bulk_load(st, g.atiles + (mb * ksl + kt) * kATile, kATile, &landed_bar[s]);
             bulk_load(st + kS_B, g.wtiles + (nb * ksl + kt) * kWTile, kWTile, &landed_bar[s]);
@@ -634,16 +648,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
       const uint32_t id_f4 = idesc_nvf4(256, 256);
       int it = 0, tcount = 0;
       bool dead = false;
-      for (int tile = pair; tile < num_tiles && !dead; tile += pairs, ++tcount) {
+      for (int item = pair; item < num_items && !dead; item += pairs, ++tcount) {
+        const int lr = item_lr(item);
         if (!mbar_wait(&acce_bar, (tcount & 1) ^ 1, abort_flag)) { give_up_both(); break; }
         tc_fence_after();
-        for (int j = 0; j < per_tile; ++j, ++it) {
+        for (int j = 0; j < lr + cpk; ++j, ++it) {
           const int s = it % kP_Stages;
           if (!mbar_wait(&ready_bar[s], (it / kP_Stages) & 1, abort_flag)) { give_up_both(); dead = true; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * kS_Size);
           const uint32_t b_addr = a_addr + kS_B;
-          if (j < g.lr_iters) {
+          if (j < lr) {
 #pragma unroll
             for (int q = 0; q < 4; ++q)
               mma_f16_pair(tbase, desc_k_sw128(a_addr + 32 * q), desc_k_sw128(b_addr + 32 * q), id_lr,
@@ -672,11 +687,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
     const uint32_t lane_base = tbase + ((uint32_t)(q * 32) << 16);
     int it = 0;
     bool dead = false;
-    for (int tile = pair; tile < num_tiles && !dead; tile += pairs) {
-      for (int j = 0; j < per_tile; ++j, ++it) {
+    for (int item = pair; item < num_items && !dead; item += pairs) {
+      const int lr = item_lr(item);
+      for (int j = 0; j < lr + cpk; ++j, ++it) {
         const int s = it % kP_Stages;
         if (!mbar_wait(&landed_bar[s], (it / kP_Stages) & 1, abort_flag)) { give_up_both(); dead = true; break; }
-        if (j >= g.lr_iters) {
+        if (j >= lr) {
           const uint8_t* st = smem + s * kS_Size;
           uint32_t wa[16], wb[32];
 #pragma unroll
@@ -711,7 +727,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
     const float alpha = g.hdr->s_gx * g.hdr->s_gw;
     uint8_t* ybuf = ychunks + (warp - 8) * kEpiChunk;
     int tcount = 0;
-    for (int tile = pair; tile < num_tiles; tile += pairs, ++tcount) {
+    for (int item = pair; item < num_items; item += pairs, ++tcount) {
+      const int tile = item / g.ks, kq = item % g.ks;
       const int mt = tile / n_tiles, nt = tile % n_tiles;
       const int col0 = nt * 256 + h * 128;
       float bl[4];   // bias of columns col0 + 32 j + lane
@@ -729,6 +746,64 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acce_leader);
       const int64_t row0 = (int64_t)mt * 256 + 128 * rank + q * 32;
+      if (g.ks > 1) {
+        // K split: this item's raw sums -> part[kq]; the warp that completes a
+        // region adds the ks partials in K order (deterministic), then applies
+        // alpha and the bias.
+        const int64_t m = row0 + lane;
+        if (m < g.M) {
+          float4* dst = reinterpret_cast<float4*>(g.part + ((size_t)kq * g.M + m) * g.N + col0);
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            dst[c] = make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
+                                 __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3]));
+        }
+        __threadfence();
+        __syncwarp();
+        int* cnt = g.cnt + (size_t)tile * 16 + rank * 8 + (warp - 8);
+        int old = 0;
+        if (lane == 0) old = atomicAdd(cnt, 1);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if (old == g.ks - 1) {
+          __threadfence();
+          // lane l reduces columns col0 + 4 l .. + 3 of every live row of the
+          // region, four rows at a time so that their loads overlap
+          const int64_t left = g.M - row0;
+          const int live = left <= 0 ? 0 : (left >= 32 ? 32 : (int)left);
+          const float4 b4 = __ldg(reinterpret_cast<const float4*>(g.bias + col0) + lane);
+          for (int r0 = 0; r0 < live; r0 += 4) {
+            float4 t[4];
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+              t[rr] = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (r0 + rr < live)
+                t[rr] = __ldcg(reinterpret_cast<const float4*>(g.part + (size_t)(row0 + r0 + rr) * g.N + col0) + lane);
+            }
+            for (int k = 1; k < g.ks; ++k) {
+#pragma unroll
+              for (int rr = 0; rr < 4; ++rr) {
+                if (r0 + rr < live) {
+                  const float4 w = __ldcg(reinterpret_cast<const float4*>(
+                                              g.part + ((size_t)k * g.M + row0 + r0 + rr) * g.N + col0) + lane);
+                  t[rr].x += w.x; t[rr].y += w.y; t[rr].z += w.z; t[rr].w += w.w;
+                }
+              }
+            }
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+              if (r0 + rr < live) {
+                const uint32_t w0 = (uint32_t)bf16_rn(fmaf(alpha, t[rr].x, b4.x)) |
+                                    ((uint32_t)bf16_rn(fmaf(alpha, t[rr].y, b4.y)) << 16);
+                const uint32_t w1 = (uint32_t)bf16_rn(fmaf(alpha, t[rr].z, b4.z)) |
+                                    ((uint32_t)bf16_rn(fmaf(alpha, t[rr].w, b4.w)) << 16);
+                *reinterpret_cast<uint2*>(g.Y + (size_t)(row0 + r0 + rr) * g.N + col0 + 4 * lane) = make_uint2(w0, w1);
+              }
+            }
+          }
+          if (lane == 0) *cnt = 0;   // ready for the next call
+        }
+        continue;
+      }
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         uint4 pk[8];
@@ -1383,6 +1458,8 @@ svdq_status launch_quantize(const svdq_params* p, const void* blob_dev, const vo
   a.hdr = reinterpret_cast<const BlobHeader*>(blob);
   a.xq = ws + W.off_xq; a.xs = ws + W.off_xs;
   a.ux = reinterpret_cast<uint16_t*>(ws + W.off_ux);
+  a.gemm_cnt = W.off_cnt > W.off_part ? reinterpret_cast<int*>(ws + W.off_cnt) : nullptr;
+  a.n_cnt = (p->N / 256) * (int)(W.Mp / 256) * 16;
   const cudaError_t e = p->fmt == SVDQ_NVFP4 ? launch_act<SVDQ_NVFP4>(p, a, W.Mp, stream)
                                              : launch_act<SVDQ_INT4_G64>(p, a, W.Mp, stream);
   if (e != cudaSuccess) return cuda_fail(e, "act_quant_kernel launch");
@@ -1413,7 +1490,15 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
     if (!make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 64, 32))
       return cuda_fail(cudaErrorInvalidValue, "tensor map encode (Y)");
     const int tiles = (N / 256) * (int)(W.Mp / 256);
-    const int pairs = std::max(1, std::min(tiles, num_sms() / 2));
+    g.ks = 1;
+    g.part = reinterpret_cast<float*>(ws + W.off_part);
+    g.cnt = reinterpret_cast<int*>(ws + W.off_cnt);
+    if (W.off_cnt > W.off_part) {   // few tokens and tiles: split K over the idle pairs
+      while (g.ks < kMaxKSplit && tiles * g.ks * 2 <= num_sms() / 2 && g.k_iters % (g.ks * 2) == 0 &&
+             g.k_iters / (g.ks * 2) >= 2)
+        g.ks *= 2;
+    }
+    const int pairs = std::max(1, std::min(tiles * g.ks, num_sms() / 2));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);
     cfg.blockDim = dim3(dev::kP_Threads);

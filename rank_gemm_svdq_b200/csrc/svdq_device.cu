@@ -174,13 +174,23 @@ __device__ __forceinline__ uint32_t pack_half2_rn(float lo, float hi) {
 // Quantise 16 consecutive smoothed activations of one token (one NVFP4
 // block, or a quarter of an INT4 group of 64 spread over 4 lanes) and store
 // codes / scales.
+// Destinations (per thread and chunk, precomputed by the caller):
+//   NVFP4: tile = this token's activation tile of the chunk's slab (null for
+//          rows past Mp), code_off / sf_off = the lane's codes and scale byte in it;
+//   INT4:  codes = the lane's 16 code bytes (null past M), sx = its group scale
+//          (null unless the lane leads its group of 4 and the row is below Mp).
+struct QuantDst {
+  uint8_t* tile;
+  uint32_t code_off, sf_off;
+  uint8_t* codes;
+  float* sx;
+};
 template <int FMT>
 // dq: NVFP4 per-code tables in shared memory, dq[e] = E4M3(e) * s_gX and
 // dq[256 + e] = its round-to-nearest reciprocal (0 where the FMA-corrected
 // division is not valid); unused for INT4.
-__device__ __forceinline__ void quantize16(const float (&xh)[16], int64_t m, int kk, const ActArgs& a,
-                                           float s_gx, float six_sg, float r6, const float* dq) {
-  const int K = a.K;
+__device__ __forceinline__ void quantize16(const float (&xh)[16], const QuantDst& dst, float six_sg, float r6,
+                                           const float* dq) {
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(xh[i]));
@@ -206,11 +216,9 @@ __device__ __forceinline__ void quantize16(const float (&xh)[16], int64_t m, int
       }
     }
     // activation tile (m / 128, slab): swizzled codes, then the slab's scale atoms
-    if (m < a.Mp) {
-      uint8_t* tile = a.xq + ((size_t)(m >> 7) * (K / 256) + kk / 256) * kATile;
-      const uint32_t rr = (uint32_t)(m & 127);
-      *reinterpret_cast<uint2*>(tile + sw128(rr, (uint32_t)(kk & 255) >> 1)) = make_uint2(p0, p1);
-      tile[kTileCodes + tile_sf(rr, (uint32_t)(kk & 255) >> 4)] = (uint8_t)e;
+    if (dst.tile) {
+      *reinterpret_cast<uint2*>(dst.tile + dst.code_off) = make_uint2(p0, p1);
+      dst.tile[dst.sf_off] = (uint8_t)e;
     }
   } else {
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // group of 64 = 4 lanes
@@ -232,10 +240,10 @@ __device__ __forceinline__ void quantize16(const float (&xh)[16], int64_t m, int
         w[i] = cvt_e4m3x2((float)q1, (float)q0);
       }
     }
-    if (m < a.M)
-      *reinterpret_cast<uint4*>(a.xq + (size_t)m * K + kk) =
+    if (dst.codes)
+      *reinterpret_cast<uint4*>(dst.codes) =
           make_uint4(w[0] | (w[1] << 16), w[2] | (w[3] << 16), w[4] | (w[5] << 16), w[6] | (w[7] << 16));
-    if (((threadIdx.x & 3) == 0) && m < a.Mp) reinterpret_cast<float*>(a.xs)[int4_sx_index(kk / 64, m, a.Mp)] = s;
+    if (dst.sx) *dst.sx = s;
   }
 }
 
@@ -285,6 +293,15 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
   const uint16_t* xrow = a.X + (live ? m : 0) * K + col;
   const int cpk = K / kActChunk / KS;      // chunks of this CTA: [c0, c0 + cpk)
   const int c0 = kidx * cpk;
+  // per-thread output locations (see QuantDst): only the chunk's offset varies
+  uint8_t* const row_tiles =
+      (FMT == SVDQ_NVFP4 && m < a.Mp) ? a.xq + (size_t)(m >> 7) * (size_t)(K / 256) * kATile : nullptr;
+  const uint32_t code_off = sw128((uint32_t)(m & 127), (uint32_t)col >> 1);
+  const uint32_t sf_off = kTileCodes + tile_sf((uint32_t)(m & 127), (uint32_t)col >> 4);
+  uint8_t* const row_codes = (FMT != SVDQ_NVFP4 && live) ? a.xq + (size_t)m * K + col : nullptr;
+  const bool sx_lead = FMT != SVDQ_NVFP4 && (lane & 3) == 0 && m < a.Mp;
+  const size_t sx_base = (size_t)(m / 128) * 256 + (size_t)(m % 128);   // int4_sx_index without the group part
+  const size_t sx_pitch = (size_t)(a.Mp / 128) * 256;
   auto load_x = [&](int c, uint4 (&x)[2]) {
     if (live && c < cpk) {
       c += c0;
@@ -353,7 +370,22 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
     float xh[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) xh[i] = __fmul_rn(half_to_f32<DT>(x16[i]), il[i]);
-    quantize16<FMT>(xh, m, kk, a, s_gx, six_sg, r6, dq_tab);
+    QuantDst qd;
+    if (FMT == SVDQ_NVFP4) {
+      qd.tile = row_tiles ? row_tiles + (size_t)(c0 + c) * kATile : nullptr;
+      qd.code_off = code_off;
+      qd.sf_off = sf_off;
+      qd.codes = nullptr;
+      qd.sx = nullptr;
+    } else {
+      qd.tile = nullptr;
+      qd.code_off = qd.sf_off = 0;
+      qd.codes = row_codes ? row_codes + (size_t)k0 : nullptr;
+      const int grp = (c0 + c) * 4 + (col >> 6);   // this lane's group of 64 (int4_sx_index)
+      qd.sx = sx_lead ? reinterpret_cast<float*>(a.xs) + (size_t)(grp >> 1) * sx_pitch + sx_base + (size_t)(grp & 1) * 128
+                      : nullptr;
+    }
+    quantize16<FMT>(xh, qd, six_sg, r6, dq_tab);
     uint4 o0, o1;
     o0.x = pack_half2_rn<DT>(xh[0], xh[1]);   o0.y = pack_half2_rn<DT>(xh[2], xh[3]);
     o0.z = pack_half2_rn<DT>(xh[4], xh[5]);   o0.w = pack_half2_rn<DT>(xh[6], xh[7]);

@@ -33,7 +33,7 @@
  * work is launched asynchronously; failures inside a kernel (a bounded wait
  * that gave up) are recorded in the status word and read by svdq_get_status.
  *
- * Constraints: K % 128 == 0 (INT4) or K % 256 == 0 (NVFP4), N % 256 == 0,
+ * Constraints: K % 256 == 0 (both formats), N % 256 == 0,
  * 0 <= rank <= 128, rank % 16 == 0,
  * M >= 0 (M = 0 is a no-op), device pointers 16-byte aligned, inputs finite.
  */

@@ -26,11 +26,11 @@ namespace {
 // ------------------------------------------------------------ parameters
 svdq_status check_params(const svdq_params* p) {
   if (!p) return SVDQ_ERR_INVALID_ARG;
-  if (p->K <= 0 || p->N <= 0 || p->K % 128 != 0 || p->N % 256 != 0) return SVDQ_ERR_INVALID_ARG;
+  // the activation kernel and the NVFP4 GEMM work in whole 256-wide K slabs
+  if (p->K <= 0 || p->N <= 0 || p->K % 256 != 0 || p->N % 256 != 0) return SVDQ_ERR_INVALID_ARG;
   if (p->rank < 0 || p->rank > 128 || p->rank % 16 != 0 || p->rank > std::min(p->K, p->N))
     return SVDQ_ERR_INVALID_ARG;
   if (p->fmt != SVDQ_INT4_G64 && p->fmt != SVDQ_NVFP4) return SVDQ_ERR_UNSUPPORTED;
-  if (p->fmt == SVDQ_NVFP4 && p->K % 256 != 0) return SVDQ_ERR_INVALID_ARG;   // whole 256-wide K slabs
   if (p->act_dtype != SVDQ_F16 && p->act_dtype != SVDQ_BF16) return SVDQ_ERR_UNSUPPORTED;
   if (!(p->alpha >= 0.0f && p->alpha <= 1.0f)) return SVDQ_ERR_INVALID_ARG;
   if (p->smooth != 0 && p->smooth != 1) return SVDQ_ERR_INVALID_ARG;

@@ -36,7 +36,7 @@ def test_status_strings():
 
 
 @pytest.mark.parametrize("bad", [dict(K=100), dict(N=100), dict(rank=8), dict(rank=-16), dict(rank=256),
-                                 dict(fmt="x"), dict(alpha=1.5), dict(K=384, fmt="nvfp4")])
+                                 dict(fmt="x"), dict(alpha=1.5), dict(K=384, fmt="nvfp4"), dict(K=384, fmt="int4")])
 def test_invalid_params_rejected(bad):
     kw = dict(K=256, N=256, rank=16, fmt="int4", dtype="bf16", alpha=0.5)
     if bad.get("fmt") == "x":
@@ -104,7 +104,7 @@ def test_prepare_matches_oracle(fmt, dtype, rank, smooth):
     tensor scales bit-exact; the truncated SVD within rounding of the
     Eckart-Young optimum the oracle's Jacobi SVD gives."""
     M, N = 96, 512
-    K = 384 if fmt == "int4" else 512
+    K = 768 if fmt == "int4" else 512
     wl = synth.custom_workload(M, K, N, rank, fmt, dtype, n_out=3, factor=60.0, smooth=smooth, seed=3)
     p = sv.params(K, N, rank, fmt, dtype, smooth=smooth)
     blob, sigma = sv.prepare(p, wl.Wt, wl.bias, wl.X)

@@ -148,3 +148,35 @@ def test_small_m_split_k(gpu, dtype, M):
     b = G.run_gpu(pp, wl.X)
     G.compare(pp, wl.X, a)
     assert np.array_equal(a.Y, b.Y)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_max_rank(gpu, fmt, dtype):
+    """Rank 128 (the largest allowed): several low-rank K-steps (up to 6 for
+    fp16's three segments) and the activation kernel's two-buffer L1 ring."""
+    wl = synth.custom_workload(200, 1024, 512, 128, fmt, dtype, n_out=8, factor=40.0, seed=77)
+    pp = G.prepare(wl)
+    run = G.run_gpu(pp, wl.X)
+    G.compare(pp, wl.X, run)
+
+
+@pytest.mark.parametrize("fmt,K", [("int4", 256), ("nvfp4", 256)])
+def test_smallest_shapes(gpu, fmt, K):
+    """One K slab and one 256-column output tile."""
+    wl = synth.custom_workload(7, K, 256, 16, fmt, "bf16", n_out=2, factor=30.0, seed=3)
+    pp = G.prepare(wl)
+    run = G.run_gpu(pp, wl.X)
+    G.compare(pp, wl.X, run)
+
+
+def test_zero_tokens_is_a_no_op(gpu):
+    import torch
+    wl = synth.custom_workload(4, 512, 512, 16, "nvfp4", "bf16", n_out=2, factor=10.0, seed=1)
+    pp = G.prepare(wl)
+    blob = torch.from_numpy(pp.blob).cuda()
+    ws = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    x = torch.empty((0, 512), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((0, 512), dtype=torch.bfloat16, device="cuda")
+    sv.linear(pp.p, blob, x, 0, y, ws)
+    assert sv.get_status() == sv.OK

@@ -191,6 +191,15 @@ svdq_status svdq_probe_div(const float* v, const float* d, int64_t n, float* q, 
                            svdq_stream stream);
 
 /*
+ * Test hook for the device-side failure path: one thread waits, with the
+ * kernels' bounded mbarrier wait, on a barrier that nothing arrives on.  After
+ * limit_ns (1 .. 2e9) it gives up and records SVDQ_ERR_TIMEOUT in the device
+ * status word, which the next svdq_get_status returns (and clears).  Nothing
+ * hangs and the context stays usable.  Asynchronous on `stream`.
+ */
+svdq_status svdq_probe_timeout(int64_t limit_ns, svdq_stream stream);
+
+/*
  * Measurement hook: tensor-core operation rate.  Launches `ctas` CTAs (pairs
  * of CTAs for op 1); in each, one thread issues `iters` back-to-back tcgen05
  * operations of kind `op` on zeroed shared memory and writes the clock64

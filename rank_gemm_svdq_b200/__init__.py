@@ -64,6 +64,7 @@ def _load():
         "svdq_probe_div": (ctypes.c_int, [vp, vp, i64, vp, vp, vp]),
         "svdq_probe_tc": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp]),
         "svdq_linear_noalloc": (ctypes.c_int, [P, vp, vp, i64, vp, vp]),
+        "svdq_probe_timeout": (ctypes.c_int, [i64, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -75,7 +76,7 @@ _lib = _load()
 EXPORTED = ("svdq_blob_bytes", "svdq_prepare", "svdq_blob_check", "svdq_blob_export",
             "svdq_workspace_bytes", "svdq_linear", "svdq_quantize_act", "svdq_gemm", "svdq_export_act", "svdq_get_status",
             "svdq_status_string", "svdq_last_error_string", "svdq_probe_cvt", "svdq_probe_div", "svdq_probe_tc",
-            "svdq_linear_noalloc")
+            "svdq_linear_noalloc", "svdq_probe_timeout")
 NOALLOC_SCRATCH_BYTES = 16 << 20   # SVDQ_NOALLOC_SCRATCH_BYTES
 
 
@@ -217,6 +218,10 @@ def probe_cvt(x, e2m1, e4m3, stream=None):
 def probe_div(v, d, q, q_ieee, stream=None):
     _check(_lib.svdq_probe_div(_ptr(v), _ptr(d), v.numel(), _ptr(q), _ptr(q_ieee), _stream(stream)),
            "svdq_probe_div")
+
+
+def probe_timeout(limit_ns: int, stream=None):
+    _check(_lib.svdq_probe_timeout(limit_ns, _stream(stream)), "svdq_probe_timeout")
 
 
 def probe_tc(op: int, iters: int, ctas: int, cycles, stream=None):

@@ -1311,6 +1311,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
   probe_body<true>(op, iters, cycles);
 }
 
+// Test hook: one thread waits, through the same bounded wait as the kernels,
+// on an mbarrier that nothing arrives on; after limit_ns it gives up and
+// records a timeout in the status word instead of hanging.
+__global__ void probe_timeout_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_sh;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_sh = 0;
+    fence_mbar_init();
+    (void)mbar_wait(&bar, 0, &abort_sh, limit_ns);
+  }
+}
+
 // Test hook: the activation kernel's quotient (reciprocal + FMA correction)
 // next to the IEEE division, on the same inputs.
 __global__ void probe_div_kernel(const float* v, const float* d, int64_t n, float* q, float* q_ieee) {
@@ -1675,6 +1689,14 @@ svdq_status svdq_probe_tc(int op, int iters, int ctas, unsigned long long* cycle
   if (op == 1 || op == 10) dev::tc_probe_pair_kernel<<<(ctas + 1) / 2 * 2, 128, dev::kProbeSmem, s>>>(op, iters, cycles);
   else dev::tc_probe_kernel<<<ctas, 256, dev::kProbeSmem, s>>>(op, iters, cycles);
   return launch_status("tc_probe launch");
+}
+
+svdq_status svdq_probe_timeout(int64_t limit_ns, svdq_stream stream) {
+  if (limit_ns <= 0 || limit_ns > 2000000000ll) return SVDQ_ERR_INVALID_ARG;
+  svdq_status st = device_ready();
+  if (st != SVDQ_OK) return st;
+  dev::probe_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>((uint64_t)limit_ns);
+  return launch_status("probe_timeout launch");
 }
 
 svdq_status svdq_probe_div(const float* v, const float* d, int64_t n, float* q, float* q_ieee,

@@ -180,3 +180,18 @@ def test_zero_tokens_is_a_no_op(gpu):
     y = torch.empty((0, 512), dtype=torch.bfloat16, device="cuda")
     sv.linear(pp.p, blob, x, 0, y, ws)
     assert sv.get_status() == sv.OK
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(gpu):
+    """A wait that nothing completes gives up after its limit, the status word
+    reports SVDQ_ERR_TIMEOUT once, and the next layer call still matches the
+    oracle (no fault, no hang)."""
+    import torch
+    assert sv.get_status() == sv.OK
+    sv.probe_timeout(50_000_000)            # 50 ms
+    torch.cuda.synchronize()
+    assert sv.get_status() == sv.ERR_TIMEOUT
+    assert sv.get_status() == sv.OK         # read and cleared
+    wl = synth.custom_workload(33, 512, 512, 16, "nvfp4", "bf16", n_out=2, factor=20.0, seed=8)
+    pp = G.prepare(wl)
+    G.compare(pp, wl.X, G.run_gpu(pp, wl.X))

@@ -12,7 +12,7 @@
 //   wq          NVFP4: weight tiles (below), [N/128][K/256] x 20480 bytes
 //               INT4:  N x K bytes, the code as an E4M3 byte (exact for -8..7)
 //   ws          NVFP4: empty (the scales live in the weight tiles)
-//               INT4:  fp32 group scales, blocked [K/128][N/256][2][256]
+//               INT4:  fp32 group scales, blocked [K/128][N/128][2][128]
 //               (one 128-wide K slab of a 256-column tile is one contiguous 2 KB)
 //   bias        N fp32
 //
@@ -157,7 +157,7 @@ SVDQ_HD inline size_t int4_sx_index(int64_t g, int64_t m, int64_t Mp) {
   return ((size_t)(g >> 1) * (size_t)(Mp / 128) + (size_t)(m / 128)) * 256 + (size_t)(g & 1) * 128 + (size_t)(m % 128);
 }
 SVDQ_HD inline size_t int4_sw_index(int64_t g, int64_t n, int64_t N) {
-  return ((size_t)(g >> 1) * (size_t)(N / 256) + (size_t)(n / 256)) * 512 + (size_t)(g & 1) * 256 + (size_t)(n % 256);
+  return ((size_t)(g >> 1) * (size_t)(N / 128) + (size_t)(n / 128)) * 256 + (size_t)(g & 1) * 128 + (size_t)(n % 128);
 }
 
 // Byte offset of (row r, byte c) inside a 128 x 128-byte tile with the 128-byte swizzle.

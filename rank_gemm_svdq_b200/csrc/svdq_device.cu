@@ -494,10 +494,7 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
 
 // ------------------------------------------------------------ kernel 2 (shared parts)
 constexpr int kBM = 128;          // tokens per tile (TMEM lanes)
-constexpr int kBN = 256;          // output features per tile (TMEM columns)
 constexpr int kABytes = kBM * 128;   // one 128-byte-wide K slab of A
-constexpr int kBBytes = kBN * 128;   // ... of B
-constexpr int kStages = 4;
 
 struct GemmArgs {
   int64_t M;
@@ -885,23 +882,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
 // scales sx[m,g] sw[n,g] cannot enter the MMA, so every group's partial is
 // drained from TMEM and folded on the CUDA cores, two columns per instruction
 // (f32x2):  acc += (P_g * sw) * sx.
-// Persistent, one CTA per SM over 128 x 256 output tiles (n fastest).
-// TMEM: two 256-column partial buffers; the MMA issuer fills one while the
-// fold warps drain the other, across tile boundaries.  The low-rank product
-// u L2 is each tile's first partial (scale 1).
-// Shared memory: a 4-deep ring of K slabs (128 bytes = two groups: A 16 KB,
-// B 32 KB, by 2D TMA), a ring of the slabs' group scales (one 1 KB and one
-// 2 KB bulk copy from the blocked scale arrays), and one 2 KB output chunk per
-// fold warp (32 rows x 32 bf16 columns, 64-byte swizzle) for TMA stores.
+// Persistent, one CTA per SM over 128 x 128 output tiles (n fastest).
+// TMEM: four 128-column partial buffers in a ring that runs across tile
+// boundaries; the MMA issuer fills one while the fold warps drain the others.
+// The hand-off (commit -> fold warps load -> release -> next MMA) has a round
+// trip of about a microsecond whatever the work, so the time it bounds is
+// (partial columns per SM / 512) x that round trip.  128-column partials keep
+// that product while letting each fold warp hold a whole share (32 rows x 64
+// columns) of a partial in registers after one load, so the buffer is
+// released before any folding arithmetic.  The low-rank product u L2 is each
+// tile's first partial (scale 1).
+// The fold reads TMEM in the 16x256b shape: a thread holds 4 rows x 16
+// columns instead of 1 row x 64, so it needs 16 column scales sw (not 64)
+// from shared memory per partial.  Broadcasting sw to every lane was the
+// kernel's bottleneck (shared-memory load wavefronts ~70 % busy) with the
+// row-per-lane shape.
+// Shared memory: a 6-deep ring of K slabs (128 bytes = two groups: A 16 KB,
+// B 16 KB, by 2D TMA), a ring of the slabs' group scales (two 1 KB bulk
+// copies from the blocked scale arrays), and one 2 KB output chunk per fold
+// warp (32 rows x 32 bf16 columns, 64-byte swizzle) for TMA stores.
 // Warps: 0 producer, 1 TMEM owner + MMA issuer, 2-3 idle [72 regs];
 // 4-11 fold / epilogue, lane quarter warp % 4, column half (warp - 4) / 4 [216]
 // (4 x 32 x 72 + 8 x 32 x 216 = the 384 x 168 registers of the launch).
-constexpr int kI4StageBytes = kABytes + kBBytes;   // A/B ring: 2 groups per stage
-constexpr int kI4ScaleSlot = 2 * kBM * 4 + 2 * kBN * 4;  // sx[2][128] + sw[2][256] fp32 = 3072
+constexpr int kI4BN = 128;                         // output features per tile
+constexpr int kI4BBytes = kI4BN * 128;             // one 128-byte-wide K slab of B
+constexpr int kI4Stages = 6;
+constexpr int kI4Bufs = 4;                         // TMEM partial buffers of kI4BN columns
+constexpr int kI4StageBytes = kABytes + kI4BBytes; // A/B ring: 2 groups per stage
+constexpr int kI4ScaleSlot = 2 * kBM * 4 + 2 * kI4BN * 4;  // sx[2][128] + sw[2][128] fp32 = 2048
 constexpr int kI4Epi = 8;
-constexpr int kI4Threads = 12 * 32;
+constexpr int kI4Threads = (4 + kI4Epi) * 32;
 constexpr int kI4Chunk = 32 * 64;                  // 32 rows x 32 bf16 columns
-constexpr int kI4Smem = kStages * (kI4StageBytes + kI4ScaleSlot) + kI4Epi * kI4Chunk + 1024;
+constexpr int kI4Smem = kI4Stages * (kI4StageBytes + kI4ScaleSlot) + kI4Epi * kI4Chunk + 1024;
+static_assert(kI4Bufs * kI4BN == 512, "the partial buffers fill TMEM");
 
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
@@ -927,27 +940,27 @@ __global__ void __launch_bounds__(kI4Threads, 1)
                      const __grid_constant__ CUtensorMap tm_ua, const __grid_constant__ CUtensorMap tm_ub,
                      const __grid_constant__ CUtensorMap tm_y, const GemmArgs g) {
   extern __shared__ __align__(1024) uint8_t gsmem_raw[];
-  __shared__ uint64_t full_bar[kStages], empty_bar[kStages], sfull_bar[kStages], sempty_bar[kStages];
-  __shared__ uint64_t pfull_bar[2], pempty_bar[2], drain_bar;
+  __shared__ uint64_t full_bar[kI4Stages], empty_bar[kI4Stages], sfull_bar[kI4Stages], sempty_bar[kI4Stages];
+  __shared__ uint64_t pfull_bar[kI4Bufs], pempty_bar[kI4Bufs], drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sring = smem + kStages * kI4StageBytes;   // scale slots
-  uint8_t* ychunks = sring + kStages * kI4ScaleSlot;
+  uint8_t* sring = smem + kI4Stages * kI4StageBytes;   // scale slots
+  uint8_t* ychunks = sring + kI4Stages * kI4ScaleSlot;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles = g.N / kBN;
+  const int n_tiles = g.N / kI4BN;
   const int num_tiles = n_tiles * (int)(g.Mp / kBM);
   const int total = g.lr_iters + g.k_iters;   // ring steps per tile
   const int has_lr = g.lr_iters > 0;
   volatile int* abort_flag = &abort_sh;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kI4Stages; ++s) {
       mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1);
       mbar_init(&sfull_bar[s], 1); mbar_init(&sempty_bar[s], kI4Epi);
     }
-    for (int b = 0; b < 2; ++b) { mbar_init(&pfull_bar[b], 1); mbar_init(&pempty_bar[b], kI4Epi); }
+    for (int b = 0; b < kI4Bufs; ++b) { mbar_init(&pfull_bar[b], 1); mbar_init(&pempty_bar[b], kI4Epi); }
     mbar_init(&drain_bar, 1);
     abort_sh = 0;
     fence_mbar_init();
@@ -970,13 +983,13 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       bool dead = false;
       for (int tile = blockIdx.x; tile < num_tiles && !dead; tile += gridDim.x) {
         const int mt = tile / n_tiles, nt = tile % n_tiles;
-        const int n0 = nt * kBN;
+        const int n0 = nt * kI4BN;
         const int64_t m0 = (int64_t)mt * kBM;
         for (int j = 0; j < total; ++j, ++it) {
-          const int s = it % kStages;
-          if (!mbar_wait(&empty_bar[s], ((it / kStages) & 1) ^ 1, abort_flag)) { dead = true; break; }
+          const int s = it % kI4Stages;
+          if (!mbar_wait(&empty_bar[s], ((it / kI4Stages) & 1) ^ 1, abort_flag)) { dead = true; break; }
           uint8_t* st = smem + s * kI4StageBytes;
-          mbar_arrive_expect_tx(&full_bar[s], kABytes + kBBytes);
+          mbar_arrive_expect_tx(&full_bar[s], kABytes + kI4BBytes);
           if (j < g.lr_iters) {
             tma_load_2d(st, &tm_ua, &full_bar[s], j * 64, (int)m0);
             tma_load_2d(st + kABytes, &tm_ub, &full_bar[s], j * 64, n0);
@@ -985,14 +998,14 @@ __global__ void __launch_bounds__(kI4Threads, 1)
             tma_load_2d(st, &tm_a, &full_bar[s], kt * 128, (int)m0);
             tma_load_2d(st + kABytes, &tm_b, &full_bar[s], kt * 128, n0);
             // the slab's two groups of scales (blocked layouts: one copy each)
-            const int ss = sk % kStages;
-            if (!mbar_wait(&sempty_bar[ss], ((sk / kStages) & 1) ^ 1, abort_flag)) { issued = it + 1; dead = true; break; }
+            const int ss = sk % kI4Stages;
+            if (!mbar_wait(&sempty_bar[ss], ((sk / kI4Stages) & 1) ^ 1, abort_flag)) { issued = it + 1; dead = true; break; }
             uint8_t* slot = sring + ss * kI4ScaleSlot;
             const float* sx = reinterpret_cast<const float*>(g.sfa) + ((size_t)kt * (size_t)(g.Mp / kBM) + mt) * 256;
-            const float* sw = reinterpret_cast<const float*>(g.sfb) + ((size_t)kt * n_tiles + nt) * 512;
+            const float* sw = reinterpret_cast<const float*>(g.sfb) + ((size_t)kt * n_tiles + nt) * (2 * kI4BN);
             mbar_arrive_expect_tx(&sfull_bar[ss], kI4ScaleSlot);
             bulk_load(slot, sx, 2 * kBM * 4, &sfull_bar[ss]);
-            bulk_load(slot + 2 * kBM * 4, sw, 2 * kBN * 4, &sfull_bar[ss]);
+            bulk_load(slot + 2 * kBM * 4, sw, 2 * kI4BN * 4, &sfull_bar[ss]);
             ++sk;
             sissued = sk;
           }
@@ -1000,41 +1013,41 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         }
       }
       if (*abort_flag) {
-        for (int i = issued - 1; i >= 0 && i >= issued - kStages; --i)
-          mbar_drain(&full_bar[i % kStages], (i / kStages) & 1);
-        for (int i = sissued - 1; i >= 0 && i >= sissued - kStages; --i)
-          mbar_drain(&sfull_bar[i % kStages], (i / kStages) & 1);
+        for (int i = issued - 1; i >= 0 && i >= issued - kI4Stages; --i)
+          mbar_drain(&full_bar[i % kI4Stages], (i / kI4Stages) & 1);
+        for (int i = sissued - 1; i >= 0 && i >= sissued - kI4Stages; --i)
+          mbar_drain(&sfull_bar[i % kI4Stages], (i / kI4Stages) & 1);
       }
     } else if (warp == 1 && lane == 0) {
-      const uint32_t id_lr = idesc_f16_bf16(kBM, kBN);
-      const uint32_t id_f8 = idesc_f8_e4m3(kBM, kBN);
+      const uint32_t id_lr = idesc_f16_bf16(kBM, kI4BN);
+      const uint32_t id_f8 = idesc_f8_e4m3(kBM, kI4BN);
       int it = 0, seq = 0;   // seq: partial-buffer sequence over all tiles
       bool dead = false;
       for (int tile = blockIdx.x; tile < num_tiles && !dead; tile += gridDim.x) {
         for (int j = 0; j < total && !dead; ++j, ++it) {
-          const int s = it % kStages;
-          if (!mbar_wait(&full_bar[s], (it / kStages) & 1, abort_flag)) { dead = true; break; }
+          const int s = it % kI4Stages;
+          if (!mbar_wait(&full_bar[s], (it / kI4Stages) & 1, abort_flag)) { dead = true; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * kI4StageBytes);
           const uint32_t b_addr = a_addr + kABytes;
           if (j < g.lr_iters) {
-            const int buf = seq & 1;
+            const int buf = seq % kI4Bufs;
             if (j == 0) {
-              if (!mbar_wait(&pempty_bar[buf], ((seq >> 1) & 1) ^ 1, abort_flag)) { dead = true; break; }
+              if (!mbar_wait(&pempty_bar[buf], ((seq / kI4Bufs) & 1) ^ 1, abort_flag)) { dead = true; break; }
               tc_fence_after();
             }
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-              mma_f16(tbase + 256 * buf, desc_k_sw128(a_addr + 32 * q), desc_k_sw128(b_addr + 32 * q), id_lr,
+              mma_f16(tbase + kI4BN * buf, desc_k_sw128(a_addr + 32 * q), desc_k_sw128(b_addr + 32 * q), id_lr,
                       (j | q) != 0);
             if (j == g.lr_iters - 1) { mma_commit(&pfull_bar[buf]); ++seq; }
           } else {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const int buf = seq & 1;
-              if (!mbar_wait(&pempty_bar[buf], ((seq >> 1) & 1) ^ 1, abort_flag)) { dead = true; break; }
+              const int buf = seq % kI4Bufs;
+              if (!mbar_wait(&pempty_bar[buf], ((seq / kI4Bufs) & 1) ^ 1, abort_flag)) { dead = true; break; }
               tc_fence_after();
-              const uint32_t d = tbase + 256 * buf;
+              const uint32_t d = tbase + kI4BN * buf;
 #pragma unroll
               for (int q = 0; q < 2; ++q)
                 mma_f8(d, desc_k_sw128(a_addr + 64 * h + 32 * q), desc_k_sw128(b_addr + 64 * h + 32 * q), id_f8,
@@ -1057,100 +1070,109 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     // fold / epilogue warps 4..11
     const int e = warp - 4;
     const int q = warp & 3;                 // TMEM lane quarter
-    const int ch = e >> 2;                  // column half
-    const int row_in_tile = q * 32 + lane;
+    const int ch = e >> 2;                  // column half of the tile
+    const int t4 = lane >> 2;               // row within an 8-row group
+    const int c2 = 2 * (lane & 3);          // column pair within an 8-column block
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     uint8_t* ybuf = ychunks + e * kI4Chunk;
     int seq = 0, sk = 0;
     bool ok = true;
-    uint64_t acc[64];   // 128 columns as f32 pairs
-    // drain partial buffer `buf` into acc: acc += (P * sw) * sx, 64 columns at a time;
-    // the buffer is released once both halves are in registers
-    auto fold = [&](int buf, const float* swp, float sxm, bool plain) {
+    // acc[8 * s + k]: rows 32q + 8s + t4 (s = 0..3), columns 64ch + 8k + c2 + {0, 1}
+    uint64_t acc[32];
+    // drain partial buffer `buf` into acc: acc += (P * sw) * sx; the buffer is
+    // released as soon as this warp's 32 x 64 share is in registers
+    auto fold = [&](int buf, const float* swp, const float* sxp, bool plain) {
+      uint32_t v[64];   // v[32 h + 4k + 2i + j]: row 16h + 8i + t4, column 8k + c2 + j
+      tmem_ld_16x256b_x8(tbase + lane_addr + kI4BN * buf + ch * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
+      tmem_ld_16x256b_x8(tbase + lane_addr + (16u << 16) + kI4BN * buf + ch * 64,
+                         *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pempty_bar[buf]);
+      if (plain) {
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t v[64];
-        tmem_ld_32cols(tbase + lane_addr + 256 * buf + ch * 128 + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
-        tmem_ld_32cols(tbase + lane_addr + 256 * buf + ch * 128 + hh * 64 + 32,
-                       *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-        tmem_ld_wait();
-        if (hh == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&pempty_bar[buf]);
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+              acc[8 * (2 * h + i) + k] =
+                  f2_pack(__uint_as_float(v[32 * h + 4 * k + 2 * i]), __uint_as_float(v[32 * h + 4 * k + 2 * i + 1]));
+      } else {
+        uint64_t sx2[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float x = sxp[8 * r + t4];
+          sx2[r] = f2_pack(x, x);
         }
-        if (plain) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) acc[hh * 32 + j] = f2_pack(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-        } else {
-          const uint64_t sx2 = f2_pack(sxm, sxm);
+        for (int k = 0; k < 8; ++k) {
+          const float2 w = *reinterpret_cast<const float2*>(swp + 8 * k + c2);
+          const uint64_t w2 = f2_pack(w.x, w.y);
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float4 w4 = *reinterpret_cast<const float4*>(swp + hh * 64 + 2 * j);
-            const uint64_t p0 = f2_mul(f2_pack(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])),
-                                       f2_pack(w4.x, w4.y));
-            const uint64_t p1 = f2_mul(f2_pack(__uint_as_float(v[2 * j + 2]), __uint_as_float(v[2 * j + 3])),
-                                       f2_pack(w4.z, w4.w));
-            acc[hh * 32 + j] = f2_fma(p0, sx2, acc[hh * 32 + j]);
-            acc[hh * 32 + j + 1] = f2_fma(p1, sx2, acc[hh * 32 + j + 1]);
-          }
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int rs = 2 * h + i;
+              const uint64_t pp = f2_mul(
+                  f2_pack(__uint_as_float(v[32 * h + 4 * k + 2 * i]), __uint_as_float(v[32 * h + 4 * k + 2 * i + 1])),
+                  w2);
+              acc[8 * rs + k] = f2_fma(pp, sx2[rs], acc[8 * rs + k]);
+            }
         }
       }
     };
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       const int mt = tile / n_tiles, nt = tile % n_tiles;
-      const int col0 = nt * kBN + ch * 128;
+      const int col0 = nt * kI4BN + ch * 64;
       const int64_t m0 = (int64_t)mt * kBM;
       if (has_lr) {
-        const int buf = seq & 1;
-        if (!mbar_wait(&pfull_bar[buf], (seq >> 1) & 1, abort_flag)) { ok = false; break; }
+        const int buf = seq % kI4Bufs;
+        if (!mbar_wait(&pfull_bar[buf], (seq / kI4Bufs) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        fold(buf, nullptr, 1.0f, true);
+        fold(buf, nullptr, nullptr, true);
         ++seq;
       } else {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) acc[j] = 0ull;
+        for (int j = 0; j < 32; ++j) acc[j] = 0ull;
       }
       for (int kt = 0; kt < g.k_iters && ok; ++kt, ++sk) {
-        const int ss = sk % kStages;
-        if (!mbar_wait(&sfull_bar[ss], (sk / kStages) & 1, abort_flag)) { ok = false; break; }
+        const int ss = sk % kI4Stages;
+        if (!mbar_wait(&sfull_bar[ss], (sk / kI4Stages) & 1, abort_flag)) { ok = false; break; }
         const float* slot = reinterpret_cast<const float*>(sring + ss * kI4ScaleSlot);
         for (int h = 0; h < 2; ++h) {
-          const int buf = seq & 1;
-          if (!mbar_wait(&pfull_bar[buf], (seq >> 1) & 1, abort_flag)) { ok = false; break; }
+          const int buf = seq % kI4Bufs;
+          if (!mbar_wait(&pfull_bar[buf], (seq / kI4Bufs) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          fold(buf, slot + 2 * kBM + h * kBN + ch * 128, slot[h * kBM + row_in_tile], false);
+          fold(buf, slot + 2 * kBM + h * kI4BN + ch * 64, slot + h * kBM + q * 32, false);
           ++seq;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sempty_bar[ss]);
       }
       if (!ok) break;
-      // epilogue: y = acc + bias -> bf16, 32-column chunks through shared memory
+      // epilogue: y = acc + bias -> bf16, two 32-column chunks through shared
+      // memory (64-byte rows, 16-byte unit u of row r stored at u ^ ((r >> 1) & 3))
       const int64_t row0 = m0 + q * 32;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float bl = __ldg(g.bias + col0 + 32 * c + lane);   // bias of column 32c + lane
-        uint4 pk[4];
+      for (int c = 0; c < 2; ++c) {
+        float2 bl[4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          uint32_t w[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int jj = 16 * c + 4 * t + i;   // f32 pair index: columns 2jj, 2jj+1
-            float y0, y1;
-            f2_unpack(acc[jj], y0, y1);
-            y0 += __shfl_sync(0xffffffffu, bl, (2 * jj) & 31);
-            y1 += __shfl_sync(0xffffffffu, bl, (2 * jj + 1) & 31);
-            w[i] = (uint32_t)bf16_rn(y0) | ((uint32_t)bf16_rn(y1) << 16);
-          }
-          pk[t] = make_uint4(w[0], w[1], w[2], w[3]);
-        }
+        for (int kk = 0; kk < 4; ++kk) bl[kk] = __ldg(reinterpret_cast<const float2*>(g.bias + col0 + 32 * c + 8 * kk + c2));
         if (lane == 0) bulk_wait_read<0>();
         __syncwarp();
 #pragma unroll
-        for (int t = 0; t < 4; ++t)
-          *reinterpret_cast<uint4*>(ybuf + lane * 64 + ((t ^ ((lane >> 1) & 3)) << 4)) = pk[t];
+        for (int rs = 0; rs < 4; ++rs) {
+          const int r = 8 * rs + t4;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            float y0, y1;
+            f2_unpack(acc[8 * rs + 4 * c + kk], y0, y1);
+            const uint32_t w = (uint32_t)bf16_rn(y0 + bl[kk].x) | ((uint32_t)bf16_rn(y1 + bl[kk].y) << 16);
+            *reinterpret_cast<uint32_t*>(ybuf + r * 64 + ((kk ^ ((r >> 1) & 3)) << 4) + 2 * c2) = w;
+          }
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && row0 < g.M) {
@@ -1562,14 +1584,14 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
   CUtensorMap tm_a, tm_b, tm_ua, tm_ub, tm_y;
   const uint64_t krow = (uint64_t)K;
   bool ok = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + W.off_xq, krow, (uint64_t)M, krow, 128, dev::kBM) &&
-            make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, blob + B.off_wq, krow, (uint64_t)N, krow, 128, dev::kBN) &&
+            make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, blob + B.off_wq, krow, (uint64_t)N, krow, 128, dev::kI4BN) &&
             make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 32, 32,
                      CU_TENSOR_MAP_SWIZZLE_64B);
   if (r > 0) {
     ok = ok && make_map(&tm_ua, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + W.off_ux, (uint64_t)lrw, (uint64_t)M,
                         (uint64_t)lrw * 2, 64, dev::kBM) &&
          make_map(&tm_ub, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, blob + B.off_l2x, (uint64_t)lrw, (uint64_t)N,
-                  (uint64_t)lrw * 2, 64, dev::kBN);
+                  (uint64_t)lrw * 2, 64, dev::kI4BN);
   } else {
     tm_ua = tm_a; tm_ub = tm_b;   // not read when rank is 0
   }
@@ -1584,7 +1606,7 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
   g.hdr = reinterpret_cast<const BlobHeader*>(blob);
   g.Y = static_cast<uint16_t*>(Y);
   g.Mp = W.Mp;
-  const int tiles = (N / dev::kBN) * (int)(W.Mp / dev::kBM);
+  const int tiles = (N / dev::kI4BN) * (int)(W.Mp / dev::kBM);
   const int grid = std::max(1, std::min(tiles, num_sms()));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);

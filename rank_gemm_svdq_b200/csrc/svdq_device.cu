@@ -112,6 +112,34 @@ __device__ __forceinline__ float div_by_recip(float v, float d, float r) {
   return __fmaf_rn(e, r, q);
 }
 
+// Two fp32 lanes per instruction (mul / fma .rn.f32x2): each lane is rounded
+// exactly as the scalar operation would be.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// div_by_recip on two lanes: v2 / d, given nd2 = (-d, -d) and r2 = (r, r).
+__device__ __forceinline__ uint64_t div2_by_recip(uint64_t v2, uint64_t nd2, uint64_t r2) {
+  const uint64_t q = f2_mul(v2, r2);
+  const uint64_t e = f2_fma(q, nd2, v2);
+  return f2_fma(e, r2, q);
+}
+
 __device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
 }
@@ -191,9 +219,12 @@ template <int FMT>
 // division is not valid); unused for INT4.
 __device__ __forceinline__ void quantize16(const float (&xh)[16], const QuantDst& dst, float six_sg, float r6,
                                            const float* dq) {
-  float amax = 0.0f;
+  float m8[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(xh[i]));
+  for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fabsf(xh[i]), fabsf(xh[i + 8]));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m8[i] = fmaxf(m8[i], m8[i + 4]);
+  float amax = fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3]));
   if constexpr (FMT == SVDQ_NVFP4) {
     const float ratio = r6 != 0.0f ? div_by_recip(amax, six_sg, r6) : __fdiv_rn(amax, six_sg);
     const uint32_t e = cvt_e4m3x2(0.0f, ratio) & 0xFFu;
@@ -202,11 +233,16 @@ __device__ __forceinline__ void quantize16(const float (&xh)[16], const QuantDst
     uint32_t p0 = 0, p1 = 0;
     if (d != 0.0f) {
       if (rd != 0.0f) {
+        const uint64_t nd2 = f2_pack(-d, -d), r2 = f2_pack(rd, rd);
+        uint32_t b[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          p0 |= cvt_e2m1x2(div_by_recip(xh[2 * i + 1], d, rd), div_by_recip(xh[2 * i], d, rd)) << (8 * i);
-          p1 |= cvt_e2m1x2(div_by_recip(xh[2 * i + 9], d, rd), div_by_recip(xh[2 * i + 8], d, rd)) << (8 * i);
+        for (int i = 0; i < 8; ++i) {
+          float q0, q1;
+          f2_unpack(div2_by_recip(f2_pack(xh[2 * i], xh[2 * i + 1]), nd2, r2), q0, q1);
+          b[i] = cvt_e2m1x2(q1, q0);
         }
+        p0 = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+        p1 = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
       } else {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -280,11 +316,11 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
   const float inv_alpha = FMT == SVDQ_NVFP4 ? 1.0f / (a.hdr->s_gx * a.hdr->s_gw) : 1.0f;
   const int n_mma = 2 * (r / 8);   // (16-token, 8-rank) tiles of u
 
-  float acc[2][4];
+  float acc[2][4], acc2[2][4];
 #pragma unroll
   for (int t = 0; t < 2; ++t)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[t][i] = 0.0f;
+    for (int i = 0; i < 4; ++i) acc[t][i] = acc2[t][i] = 0.0f;
 
   const int rw = warp * 2 + (lane >> 4);     // token row inside the CTA
   const int64_t m = m0 + rw;
@@ -369,7 +405,10 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
     const uint16_t* x16 = reinterpret_cast<const uint16_t*>(xc);
     float xh[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) xh[i] = __fmul_rn(half_to_f32<DT>(x16[i]), il[i]);
+    for (int i = 0; i < 8; ++i)
+      f2_unpack(f2_mul(f2_pack(half_to_f32<DT>(x16[2 * i]), half_to_f32<DT>(x16[2 * i + 1])),
+                       f2_pack(il[2 * i], il[2 * i + 1])),
+                xh[2 * i], xh[2 * i + 1]);
     QuantDst qd;
     if (FMT == SVDQ_NVFP4) {
       qd.tile = row_tiles ? row_tiles + (size_t)(c0 + c) * kATile : nullptr;
@@ -407,12 +446,16 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
         const int mt = tt & 1, nt = tt >> 1;
         const uint32_t a_base = smem_u32(xs16(buf) + (mt * 16 + (lane & 15)) * kActStride + (lane >> 4) * 8);
         const uint32_t b_base = smem_u32(l1c + (nt * 8 + (lane & 7)) * kActStride + ((lane >> 3) & 1) * 8);
+        // two accumulators (even / odd k-steps) halve the dependent MMA chain
 #pragma unroll 4
-        for (int ks = 0; ks < kActChunk / 16; ++ks) {
+        for (int ks = 0; ks < kActChunk / 16; ks += 2) {
           uint32_t a0, a1, a2, a3, b0, b1;
           ldmatrix_x4(a_base + ks * 32, a0, a1, a2, a3);
           ldmatrix_x2(b_base + ks * 32, b0, b1);
           mma_16816<DT>(acc[t], a0, a1, a2, a3, b0, b1);
+          ldmatrix_x4(a_base + ks * 32 + 32, a0, a1, a2, a3);
+          ldmatrix_x2(b_base + ks * 32 + 32, b0, b1);
+          mma_16816<DT>(acc2[t], a0, a1, a2, a3, b0, b1);
         }
       }
     }
@@ -420,6 +463,10 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
     xn[0] = xnn[0]; xn[1] = xnn[1];
   }
   cp_async_wait_all();
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[t][i] += acc2[t][i];
   if (KS > 1) {
     // partial u of this CTA -> its shared memory; CTA 0 adds ranks 1..ks-1 in order
     float* red = reinterpret_cast<float*>(act_smem);
@@ -915,25 +962,6 @@ constexpr int kI4Threads = (4 + kI4Epi) * 32;
 constexpr int kI4Chunk = 32 * 64;                  // 32 rows x 32 bf16 columns
 constexpr int kI4Smem = kI4Stages * (kI4StageBytes + kI4ScaleSlot) + kI4Epi * kI4Chunk + 1024;
 static_assert(kI4Bufs * kI4BN == 512, "the partial buffers fill TMEM");
-
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
 
 __global__ void __launch_bounds__(kI4Threads, 1)
     gemm_int4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,

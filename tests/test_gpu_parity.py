@@ -195,3 +195,21 @@ def test_bounded_wait_reports_timeout_and_context_survives(gpu):
     wl = synth.custom_workload(33, 512, 512, 16, "nvfp4", "bf16", n_out=2, factor=20.0, seed=8)
     pp = G.prepare(wl)
     G.compare(pp, wl.X, G.run_gpu(pp, wl.X))
+
+
+@pytest.mark.parametrize("M,K,N,rank,dtype", [
+    (2, 4096, 512, 0, "bf16"),      # K split over 8 CTA pairs, no low-rank branch
+    (6, 4096, 512, 32, "fp16"),     # three low-rank segments
+    (8, 2048, 1024, 32, "bf16"),
+    (3, 4096, 9728, 16, "bf16"),    # 38 output tiles: just past the K-split limit
+])
+def test_few_token_path(gpu, M, K, N, rank, dtype):
+    """A handful of tokens (the decode-like VAR steps): codes bit-exact, Y
+    against the oracle, and two calls give identical bits (K-split partials
+    are added in K order)."""
+    wl = synth.custom_workload(M, K, N, rank, "nvfp4", dtype, n_out=6, factor=60.0, seed=90 + M)
+    pp = G.prepare(wl)
+    a = G.run_gpu(pp, wl.X)
+    b = G.run_gpu(pp, wl.X)
+    G.compare(pp, wl.X, a)
+    assert np.array_equal(a.Y, b.Y)

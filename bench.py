@@ -154,18 +154,23 @@ def device_smi_id(torch, dev):
         return vis.split(",")[dev] if vis else str(dev)
 
 
-def oracle_layer(wl):
+def oracle_layer(wl, X_cal=None):
     """The CPU oracle's layer, built from the library's host-prepared factors
-    (the offline SVD is not part of the timed linear)."""
+    (the offline SVD is not part of the timed linear).  X_cal: calibration
+    activations (default: the workload's own)."""
     import rank_gemm_svdq_b200 as sv
     import synth
     from oracle import svdquant as sq
+    X_cal = wl.X if X_cal is None else X_cal
     p = sv.params(wl.K, wl.N, wl.rank, wl.fmt, wl.dtype, wl.alpha, wl.smooth)
-    blob, _ = sv.prepare(p, wl.Wt, wl.bias, wl.X)
+    blob, _ = sv.prepare(p, wl.Wt, wl.bias, X_cal)
     c = sv.blob_export(p, blob)
-    L1, L2 = synth.bf16_bits_to_f64(c.L1), synth.bf16_bits_to_f64(c.L2)
-    return sq.prepare(wl.x_f64(), wl.Wt, wl.bias, wl.rank, wl.fmt, wl.dtype, wl.alpha, wl.smooth,
-                      factors=(c.inv_lambda, L1, L2))
+    if wl.dtype == "fp16":
+        L1, L2 = c.L1.view(np.float16).astype(np.float64), c.L2.view(np.float16).astype(np.float64)
+    else:
+        L1, L2 = synth.bf16_bits_to_f64(c.L1), synth.bf16_bits_to_f64(c.L2)
+    return sq.prepare(synth.dtype_to_f64(X_cal, wl.dtype), wl.Wt, wl.bias, wl.rank, wl.fmt, wl.dtype, wl.alpha,
+                      wl.smooth, factors=(c.inv_lambda, L1, L2))
 
 
 def blas_threads():
@@ -215,24 +220,69 @@ def max_over_ranks(value, dist, device):
 
 
 def config_dict(wl, extra=None):
-    d = {"workload": f"{WORKLOAD}: FLUX.1-like FFN up projection M={wl.M} K={wl.K} N={wl.N} rank={wl.rank} "
-                     f"NVFP4 (E2M1, E4M3/16, fp32 tensor scale), bf16 X, 1% outlier channels x50",
-         "M": wl.M, "K": wl.K, "N": wl.N, "rank": wl.rank, "format": "nvfp4", "act_dtype": "bf16",
-         "l2": "flushed by a 256 MiB write before every timed step"}
+    if wl.name == WORKLOAD:
+        desc = (f"{WORKLOAD}: FLUX.1-like FFN up projection M={wl.M} K={wl.K} N={wl.N} rank={wl.rank} "
+                f"NVFP4 (E2M1, E4M3/16, fp32 tensor scale), bf16 X, 1% outlier channels x50")
+    else:
+        desc = f"{wl.name}: M={wl.M} K={wl.K} N={wl.N} rank={wl.rank} {wl.fmt} {wl.dtype} X"
+    d = {"workload": desc, "M": wl.M, "K": wl.K, "N": wl.N, "rank": wl.rank, "format": wl.fmt,
+         "act_dtype": wl.dtype, "l2": "flushed by a 256 MiB write before every timed step"}
     if extra:
         d.update(extra)
     return d
+
+
+def gemm_roofline(wl, ms_gemm, ms_act, peaks):
+    """Roofline of the GEMM kernel.  Below the ridge (~1380 flop/B for FP4,
+    ~690 for E4M3-coded INT4: M <= 256 here) it is bound by HBM: algorithmic
+    bytes against the measured copy bandwidth.  Above it, by the tensor
+    cores: against the measured burst cuBLAS bf16 rate times the nominal dense
+    ratio of the MMA kind (FP4 x4, FP8 x2)."""
+    M, K, N, r = wl.M, wl.K, wl.N, wl.rank
+    nvfp4 = wl.fmt == "nvfp4"
+    kernel = "gemm_nvfp4_pair_kernel" if nvfp4 else "gemm_int4_kernel"
+    gemm_flops = flops(M, K, N, r)
+    alg_bytes = gemm_alg_bytes(M, K, N, r, wl.fmt)
+    common = {"kernel": kernel, "alg_flops_per_launch": gemm_flops, "alg_bytes_per_launch": alg_bytes,
+              "traffic": profiled_traffic() if wl.name == WORKLOAD and not wl.info.get("sliced") else None,
+              "kernel_ms": {"gemm": ms_gemm, "act_quant": ms_act}}
+    if M <= 256:
+        achieved = alg_bytes / (ms_gemm * 1e-3) / 1e9
+        if peaks and "hbm_gbs" in peaks:
+            peak, note = float(peaks["hbm_gbs"]), f"of measured: copy bandwidth {peaks['hbm_gbs']} GB/s"
+        else:
+            peak, note = 6650.0, "of fallback: 6.65 TB/s"
+        return dict(bound="hbm", achieved=achieved, peak=peak, unit="GB/s", frac=achieved / peak,
+                    peak_source=note, **common)
+    ratio = (NOMINAL_FP4_TFLOPS if nvfp4 else 4500.0) / NOMINAL_BF16_TFLOPS
+    # The timed loop lasts tens of milliseconds at full clocks, so the GEMM is
+    # compared with the burst (not the power-capped sustained) cuBLAS figure.
+    if peaks and "bf16_tflops" in peaks:
+        peak = float(peaks["bf16_tflops"]) * ratio
+        note = (f"of measured: burst cuBLAS bf16 {peaks['bf16_tflops']} TFLOP/s x {ratio:g} "
+                f"(nominal dense {'FP4' if nvfp4 else 'FP8'}/BF16 ratio)")
+    else:
+        peak, note = 1590.0 * ratio, f"of fallback: 1.59 PFLOP/s burst bf16 x {ratio:g}"
+    achieved = gemm_flops / (ms_gemm * 1e-3) / 1e12
+    out = dict(bound="tensor", achieved=achieved, peak=peak, unit="TFLOP/s", frac=achieved / peak,
+               peak_source=note, **common)
+    if nvfp4:
+        out["frac_of_nominal_fp4"] = achieved / NOMINAL_FP4_TFLOPS
+    return out
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
     import synth
-    wl = synth.make_workload(WORKLOAD)
+    wl = synth.make_workload(args.workload)
     ref = oracle_layer(wl)
     from oracle import svdquant as sq
+    if args.tokens:
+        wl.X = np.ascontiguousarray(wl.X[:args.tokens])
+        wl.M = args.tokens
     x = wl.x_f64()
-    S = 256
+    S = min(256, wl.M)
     times = []
     for it in range(args.warmup + args.steps):
         rows = slice((it * S) % wl.M, (it * S) % wl.M + S)
@@ -260,6 +310,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="another synthetic layer preset (synth.PRESETS); the default is the headline layer")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run on the first M tokens of the workload (calibration still uses all of them)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -286,13 +340,21 @@ def main():
         if dist is not None:
             dist.barrier()
 
-    wl = synth.make_workload(WORKLOAD, seed=0)
+    wl = synth.make_workload(args.workload, seed=0)
+    X_cal = wl.X
+    if args.tokens:
+        wl.X = np.ascontiguousarray(wl.X[:args.tokens])
+        wl.M = args.tokens
+        wl.info["sliced"] = True
     wl.X = replica_batch(wl, rank)
+    if not args.tokens:
+        X_cal = wl.X
     p = sv.params(wl.K, wl.N, wl.rank, wl.fmt, wl.dtype, wl.alpha, wl.smooth)
-    blob_host, _ = sv.prepare(p, wl.Wt, wl.bias, wl.X)
+    blob_host, _ = sv.prepare(p, wl.Wt, wl.bias, X_cal)
     dev = torch.device("cuda", local)
     blob = torch.from_numpy(blob_host).to(dev)
-    X = torch.from_numpy(wl.X.view(np.int16)).to(dev).view(torch.bfloat16)
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float16
+    X = torch.from_numpy(wl.X.view(np.int16)).to(dev).view(tdt)
     Y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=dev)
     ws = torch.empty(sv.workspace_bytes(p, wl.M), dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -356,7 +418,7 @@ def main():
     # three streams (copy in / compute / copy out) with two device buffer sets,
     # so one step's transfers overlap its neighbours' work, as a serving loop
     # would run; the time is first copy-in to last copy-out, over all steps.
-    Xh = torch.from_numpy(wl.X.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Xh = torch.from_numpy(wl.X.view(np.int16)).view(tdt).pin_memory()
     Yh = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     Xd = [torch.empty_like(X) for _ in range(2)]
     Yd = [Y, torch.empty_like(Y)]
@@ -395,35 +457,18 @@ def main():
     e2e_value = flops(M, K, N, r) * world / (e_total / esteps * 1e-3) / 1e12
     assert sv.get_status() == sv.OK
 
-    peaks = measured_peaks()
-    # The timed loop lasts tens of milliseconds at full clocks, so the GEMM is
-    # compared with the burst (not the power-capped sustained) cuBLAS figure.
-    if peaks and "bf16_tflops" in peaks:
-        peak = float(peaks["bf16_tflops"]) * (NOMINAL_FP4_TFLOPS / NOMINAL_BF16_TFLOPS)
-        peak_note = ("of measured: burst cuBLAS bf16 "
-                     f"{peaks['bf16_tflops']} TFLOP/s x 4 (nominal dense FP4/BF16 ratio)")
-    else:
-        peak = 1590.0 * 4
-        peak_note = "of fallback: 1.59 PFLOP/s burst bf16 x 4"
-    gemm_flops = flops(M, K, N, r)
-    achieved = gemm_flops / (ms_gemm * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "gemm_nvfp4_pair_kernel", "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": profiled_traffic(), "peak_source": peak_note,
-                "frac_of_nominal_fp4": achieved / NOMINAL_FP4_TFLOPS,
-                "alg_flops_per_launch": gemm_flops,
-                "alg_bytes_per_launch": gemm_alg_bytes(M, K, N, r, "nvfp4"),
-                "kernel_ms": {"gemm": ms_gemm, "act_quant": ms_act}}
+    roofline = gemm_roofline(wl, ms_gemm, ms_act, measured_peaks())
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+            "vs_baseline": None, "dtype": wl.fmt, "data": "synthetic",
             "config": config_dict(wl, {"parallelism": f"replicas x{world} (token batches, no collective)"}),
             "roofline": roofline, "clocks": clocks, "gpu_launches": 2 * args.steps,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(X.numel() * 2),
                     "d2h_bytes_per_step": int(Y.numel() * 2)},
             "frac_of_nominal_fp4": value / NOMINAL_FP4_TFLOPS}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, oracle_layer(wl))
+        line["cpu_baseline"] = cpu_baseline(wl, oracle_layer(wl, X_cal))
     if dist is not None:
         barrier()
         dist.destroy_process_group()

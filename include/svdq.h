@@ -119,6 +119,27 @@ svdq_status svdq_blob_export(const svdq_params* p, const void* blob, float* inv_
                              uint16_t* L1, uint16_t* L2, uint8_t* wcodes, void* wscales,
                              float* tscales, float* bias);
 
+/*
+ * Add a LoRA branch to a prepared layer without re-quantising it
+ * ("SVDQuant是什么？" 概述简介 and 功能特色, LoRA集成: off-the-shelf low-rank
+ * adapters plug into the quantised model with no new quantisation).  The
+ * layer then computes Y' = Y + X A B.  Since X = X^ diag(lambda), the
+ * adapter joins the 16-bit low-rank branch:
+ *   L1' = [L1 | act_dtype(lambda_eff (.) A)]   K x (r + r_lora),
+ *   L2' = [L2 ; act_dtype(B)]                  (r + r_lora) x N,
+ * with lambda_eff_j = 1 / inv_lambda_j as stored; the 4-bit residual, its
+ * scales, lambda, the tensor scales and the bias are copied unchanged.
+ * A: K x r_lora fp32 host (row-major); B: r_lora x N fp32 host (any LoRA
+ * scaling already folded in).  r_lora > 0, r_lora % 16 == 0 and
+ * p->rank + r_lora <= 128, else SVDQ_ERR_INVALID_ARG.  blob_in (blob_in_bytes,
+ * checked as by svdq_blob_check) is read only; blob_out is a host buffer of
+ * blob_out_bytes >= svdq_blob_bytes(p_out), written in full; *p_out receives
+ * p with rank = p->rank + r_lora.  Adapters stack by calling it again.
+ */
+svdq_status svdq_append_lora(const svdq_params* p, const void* blob_in, size_t blob_in_bytes, const float* A,
+                             const float* B, int32_t r_lora, svdq_params* p_out, void* blob_out,
+                             size_t blob_out_bytes);
+
 /* Device workspace bytes svdq_linear needs for M tokens. */
 size_t svdq_workspace_bytes(const svdq_params* p, int64_t M);
 

@@ -153,6 +153,20 @@ def prepare(x_cal, Wt, bias, rank, fmt, dtype, alpha=0.5, smooth=True, group=64,
     return Prepared(fmt, dtype, L1.shape[1], inv_lambda, lam_eff, L1, L2, sigma, R, wq, s_gx, b)
 
 
+def append_lora(p: Prepared, A: np.ndarray, B: np.ndarray) -> Prepared:
+    """A LoRA adapter X A B added to a prepared layer with no re-quantisation
+    ("SVDQuant是什么？…" 概述简介 and 功能特色, LoRA集成).  Reading: the adapter
+    joins the 16-bit branch.  X = X^ diag(lambda), so X A B = X^ (diag(lambda) A) B:
+    L1 gains the columns dtype(lambda_eff A) and L2 the rows dtype(B); the
+    residual R, its codes and scales, lambda and the bias stay as they are."""
+    A = np.asarray(A, dtype=np.float64)
+    B = np.asarray(B, dtype=np.float64)
+    L1 = np.hstack([p.L1, formats.to_dtype(p.lam_eff[:, None] * A, p.dtype)])
+    L2 = np.vstack([p.L2, formats.to_dtype(B, p.dtype)])
+    return Prepared(p.fmt, p.dtype, p.rank + A.shape[1], p.inv_lambda, p.lam_eff, L1, L2, p.sigma, p.R, p.wq,
+                    p.s_gx, p.bias)
+
+
 # ----------------------------------------------------------------- online side
 def smooth_act(x: np.ndarray, inv_lambda: np.ndarray) -> np.ndarray:
     """X^ = fp32(x) * inv_lambda, one fp32 multiply per element."""

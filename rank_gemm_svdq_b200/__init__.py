@@ -52,6 +52,7 @@ def _load():
         "svdq_prepare": (ctypes.c_int, [P, vp, vp, vp, i64, vp, sz, vp]),
         "svdq_blob_check": (ctypes.c_int, [P, vp, sz]),
         "svdq_blob_export": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "svdq_append_lora": (ctypes.c_int, [P, vp, sz, vp, vp, ctypes.c_int32, P, vp, sz]),
         "svdq_workspace_bytes": (sz, [P, i64]),
         "svdq_linear": (ctypes.c_int, [P, vp, vp, i64, vp, vp, sz, vp]),
         "svdq_quantize_act": (ctypes.c_int, [P, vp, vp, i64, vp, sz, vp]),
@@ -73,7 +74,7 @@ def _load():
 
 
 _lib = _load()
-EXPORTED = ("svdq_blob_bytes", "svdq_prepare", "svdq_blob_check", "svdq_blob_export",
+EXPORTED = ("svdq_blob_bytes", "svdq_prepare", "svdq_blob_check", "svdq_blob_export", "svdq_append_lora",
             "svdq_workspace_bytes", "svdq_linear", "svdq_quantize_act", "svdq_gemm", "svdq_export_act", "svdq_get_status",
             "svdq_status_string", "svdq_last_error_string", "svdq_probe_cvt", "svdq_probe_div", "svdq_probe_tc",
             "svdq_linear_noalloc", "svdq_probe_timeout")
@@ -147,6 +148,21 @@ class BlobContents:
     s_gx: np.float32
     s_gw: np.float32
     bias: np.ndarray
+
+
+def append_lora(p: svdq_params, blob: np.ndarray, A: np.ndarray, B: np.ndarray):
+    """Blob with the LoRA branch X A B added (A: K x r_lora, B: r_lora x N);
+    returns (params with the larger rank, new blob)."""
+    A = np.ascontiguousarray(A, dtype=np.float32)
+    B = np.ascontiguousarray(B, dtype=np.float32)
+    r_lora = A.shape[1]
+    assert A.shape == (p.K, r_lora) and B.shape == (r_lora, p.N)
+    q = svdq_params(p.K, p.N, p.rank + r_lora, p.fmt, p.act_dtype, p.smooth, p.alpha, 0)
+    out = np.zeros(max(blob_bytes(q), 1), np.uint8)
+    p_out = svdq_params()
+    _check(_lib.svdq_append_lora(ctypes.byref(p), _ptr(blob), blob.nbytes, _ptr(A), _ptr(B), r_lora,
+                                 ctypes.byref(p_out), _ptr(out), out.nbytes), "svdq_append_lora")
+    return p_out, out
 
 
 def blob_export(p: svdq_params, blob: np.ndarray) -> BlobContents:

@@ -345,6 +345,64 @@ uint64_t fnv1a(const uint8_t* p, size_t n) {
   return h;
 }
 
+// Write the low-rank factors (act_dtype values, as doubles) in their device
+// layouts: l1t = L1^T (r x K), and l2x, the N x lrw B operand of the up
+// projection, [L2 ; L2] for bf16 X or [L2h ; L2h ; L2l] for fp16 X (L2 =
+// L2h + L2l exactly), row-major (INT4) or as swizzled low-rank tiles (NVFP4).
+void write_factors(const svdq_params* p, const BlobLayout& L, uint8_t* base, const double* L1, const double* L2) {
+  const int K = p->K, N = p->N, r = p->rank, dt = p->act_dtype;
+  uint16_t* l1t = (uint16_t*)(base + L.off_l1t);
+  for (int i = 0; i < r; ++i)
+    for (int j = 0; j < K; ++j) l1t[(size_t)i * K + j] = dtype_bits(L1[(size_t)j * r + i], dt);
+  uint16_t* l2x = (uint16_t*)(base + L.off_l2x);
+  const int w2 = lr_width(*p);
+  auto l2x_at = [&](int n, int e) -> uint16_t& {
+    if (p->fmt != SVDQ_NVFP4) return l2x[(size_t)n * w2 + e];
+    uint8_t* tile = base + L.off_l2x + ((size_t)(n / 128) * (w2 / 64) + e / 64) * kLRTile;
+    return *reinterpret_cast<uint16_t*>(tile + sw128(n % 128, (e % 64) * 2));
+  };
+  for (int n = 0; n < N; ++n)
+    for (int i = 0; i < r; ++i) {
+      const double v = L2[(size_t)i * N + n];
+      const double hi = bf16_round(v), lo = v - hi;                  // lo exact in bf16
+      l2x_at(n, i) = bf16_bits_exact(hi);
+      l2x_at(n, r + i) = bf16_bits_exact(hi);
+      if (L.nseg == 3) l2x_at(n, 2 * r + i) = bf16_bits_exact(lo);
+    }
+}
+
+// Read the low-rank factors back as act_dtype values (the inverse of write_factors).
+void read_factors(const svdq_params* p, const BlobLayout& L, const uint8_t* base, double* L1, double* L2) {
+  const int K = p->K, N = p->N, r = p->rank, dt = p->act_dtype;
+  const uint16_t* l1t = (const uint16_t*)(base + L.off_l1t);
+  for (int j = 0; j < K; ++j)
+    for (int i = 0; i < r; ++i) L1[(size_t)j * r + i] = dtype_value(l1t[(size_t)i * K + j], dt);
+  const uint16_t* l2x = (const uint16_t*)(base + L.off_l2x);
+  const int w2 = lr_width(*p);
+  auto at = [&](int n, int e) -> uint16_t {
+    if (p->fmt != SVDQ_NVFP4) return l2x[(size_t)n * w2 + e];
+    const uint8_t* tile = base + L.off_l2x + ((size_t)(n / 128) * (w2 / 64) + e / 64) * kLRTile;
+    return *reinterpret_cast<const uint16_t*>(tile + sw128(n % 128, (e % 64) * 2));
+  };
+  for (int i = 0; i < r; ++i)
+    for (int n = 0; n < N; ++n) {
+      double v = bf16_value(at(n, i));
+      if (L.nseg == 3) v += bf16_value(at(n, 2 * r + i));
+      L2[(size_t)i * N + n] = v;
+    }
+}
+
+void finish_header(const svdq_params* p, const BlobLayout& L, uint8_t* base) {
+  BlobHeader* h = (BlobHeader*)base;
+  h->magic0 = kMagic0; h->magic1 = kMagic1; h->version = kVersion; h->header_bytes = (uint32_t)kAlign;
+  h->params = *p;
+  h->total_bytes = L.total;
+  h->off_inv_lambda = L.off_inv_lambda; h->off_l1t = L.off_l1t; h->off_l2x = L.off_l2x;
+  h->off_wq = L.off_wq; h->off_ws = L.off_ws; h->off_bias = L.off_bias;
+  h->nseg = L.nseg;
+  h->checksum = fnv1a(base + kAlign, L.total - kAlign);
+}
+
 }  // namespace
 
 // ======================================================================= C ABI
@@ -493,36 +551,12 @@ svdq_status svdq_prepare(const svdq_params* p, const float* Wt, const float* bia
   }
 
   // --- 6. factors in device layouts
-  uint16_t* l1t = (uint16_t*)(base + L.off_l1t);
-  for (int i = 0; i < r; ++i)
-    for (int j = 0; j < K; ++j) l1t[(size_t)i * K + j] = dtype_bits(L1[(size_t)j * r + i], dt);
-  uint16_t* l2x = (uint16_t*)(base + L.off_l2x);
-  const int w2 = lr_width(*p);
-  // element (n, e) of the N x w2 low-rank B operand: row-major (INT4) or tiles (NVFP4)
-  auto l2x_at = [&](int n, int e) -> uint16_t& {
-    if (p->fmt != SVDQ_NVFP4) return l2x[(size_t)n * w2 + e];
-    uint8_t* tile = base + L.off_l2x + ((size_t)(n / 128) * (w2 / 64) + e / 64) * kLRTile;
-    return *reinterpret_cast<uint16_t*>(tile + sw128(n % 128, (e % 64) * 2));
-  };
-  for (int n = 0; n < N; ++n)
-    for (int i = 0; i < r; ++i) {
-      const double v = L2[(size_t)i * N + n];
-      const double hi = bf16_round(v), lo = v - hi;                  // lo exact in bf16
-      l2x_at(n, i) = bf16_bits_exact(hi);
-      l2x_at(n, r + i) = bf16_bits_exact(hi);
-      if (L.nseg == 3) l2x_at(n, 2 * r + i) = bf16_bits_exact(lo);
-    }
+  write_factors(p, L, base, L1.data(), L2.data());
   float* bb = (float*)(base + L.off_bias);
   for (int n = 0; n < N; ++n) bb[n] = bias ? bias[n] : 0.0f;
 
   // --- 7. header
-  h->magic0 = kMagic0; h->magic1 = kMagic1; h->version = kVersion; h->header_bytes = (uint32_t)kAlign;
-  h->params = *p;
-  h->total_bytes = L.total;
-  h->off_inv_lambda = L.off_inv_lambda; h->off_l1t = L.off_l1t; h->off_l2x = L.off_l2x;
-  h->off_wq = L.off_wq; h->off_ws = L.off_ws; h->off_bias = L.off_bias;
-  h->nseg = L.nseg;
-  h->checksum = fnv1a(base + kAlign, L.total - kAlign);
+  finish_header(p, L, base);
   return SVDQ_OK;
 }
 
@@ -607,6 +641,51 @@ svdq_status svdq_blob_export(const svdq_params* p, const void* blob, float* inv_
   }
   if (tscales) { tscales[0] = h->s_gx; tscales[1] = h->s_gw; }
   if (bias) memcpy(bias, base + L.off_bias, (size_t)N * 4);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_append_lora(const svdq_params* p, const void* blob_in, size_t blob_in_bytes, const float* A,
+                             const float* B, int32_t r_lora, svdq_params* p_out, void* blob_out,
+                             size_t blob_out_bytes) {
+  svdq_status st = svdq_blob_check(p, blob_in, blob_in_bytes);
+  if (st != SVDQ_OK) return st;
+  if (!A || !B || !p_out || !blob_out || r_lora <= 0 || r_lora % 16 != 0 || p->rank + r_lora > 128)
+    return SVDQ_ERR_INVALID_ARG;
+  svdq_params q = *p;
+  q.rank = p->rank + r_lora;
+  if ((st = check_params(&q)) != SVDQ_OK) return st;
+  const BlobLayout Li = blob_layout(*p), Lo = blob_layout(q);
+  if (blob_out_bytes < Lo.total) return SVDQ_ERR_INVALID_ARG;
+  const int K = p->K, N = p->N, r = p->rank, r2 = q.rank, dt = p->act_dtype;
+  const uint8_t* in = (const uint8_t*)blob_in;
+  uint8_t* out = (uint8_t*)blob_out;
+
+  // L1' = [L1 | dtype(lambda_eff (.) A)], L2' = [L2 ; dtype(B)], since X A B = X^ (diag(lambda) A) B
+  std::vector<double> L1((size_t)K * r), L2((size_t)r * N);
+  read_factors(p, Li, in, L1.data(), L2.data());
+  const float* inv_lambda = (const float*)(in + Li.off_inv_lambda);
+  std::vector<double> L1o((size_t)K * r2), L2o((size_t)r2 * N);
+  for (int j = 0; j < K; ++j) {
+    const double lam = 1.0 / (double)inv_lambda[j];
+    for (int i = 0; i < r; ++i) L1o[(size_t)j * r2 + i] = L1[(size_t)j * r + i];
+    for (int i = 0; i < r_lora; ++i)
+      L1o[(size_t)j * r2 + r + i] = dtype_round(lam * (double)A[(size_t)j * r_lora + i], dt);
+  }
+  for (int i = 0; i < r; ++i)
+    for (int n = 0; n < N; ++n) L2o[(size_t)i * N + n] = L2[(size_t)i * N + n];
+  for (int i = 0; i < r_lora; ++i)
+    for (int n = 0; n < N; ++n) L2o[(size_t)(r + i) * N + n] = dtype_round((double)B[(size_t)i * N + n], dt);
+
+  // everything else is carried over unchanged: the residual is not re-quantised
+  memset(out, 0, Lo.total);
+  memcpy(out, in, sizeof(BlobHeader));
+  memcpy(out + Lo.off_inv_lambda, in + Li.off_inv_lambda, (size_t)K * 4);
+  memcpy(out + Lo.off_wq, in + Li.off_wq, Li.off_ws - Li.off_wq);
+  memcpy(out + Lo.off_ws, in + Li.off_ws, Li.off_bias - Li.off_ws);
+  memcpy(out + Lo.off_bias, in + Li.off_bias, (size_t)N * 4);
+  write_factors(&q, Lo, out, L1o.data(), L2o.data());
+  finish_header(&q, Lo, out);
+  *p_out = q;
   return SVDQ_OK;
 }
 

@@ -27,7 +27,7 @@ _GOLDEN = np.uint64(0x9E3779B97F4A7C15)
 _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
 
-TAGS = {"X": 1, "W": 2, "outlier": 3, "bias": 4, "gelu": 5, "extra": 6}
+TAGS = {"X": 1, "W": 2, "outlier": 3, "bias": 4, "gelu": 5, "extra": 6, "lora_A": 7, "lora_B": 8}
 
 
 def _mix(z: np.ndarray) -> np.ndarray:
@@ -181,6 +181,13 @@ def make_weight(seed: int, N: int, K: int) -> np.ndarray:
 
 def make_bias(seed: int, N: int) -> np.ndarray:
     return normal(seed, "bias", N).astype(np.float32)
+
+
+def make_lora(seed: int, K: int, N: int, r: int) -> tuple[np.ndarray, np.ndarray]:
+    """A LoRA adapter: A (K x r) fp32 ~ N(0, 1/sqrt(K)), B (r x N) fp32 ~ N(0, 0.5/sqrt(r))."""
+    A = (normal(seed, "lora_A", K * r) / math.sqrt(K)).astype(np.float32).reshape(K, r)
+    B = (normal(seed, "lora_B", r * N) * (0.5 / math.sqrt(r))).astype(np.float32).reshape(r, N)
+    return A, B
 
 
 # Workloads.  Shapes and distributions of the pages' layers; no dataset or

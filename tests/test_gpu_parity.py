@@ -213,3 +213,16 @@ def test_few_token_path(gpu, M, K, N, rank, dtype):
     b = G.run_gpu(pp, wl.X)
     G.compare(pp, wl.X, a)
     assert np.array_equal(a.Y, b.Y)
+
+
+@pytest.mark.parametrize("fmt,dtype,M", [("nvfp4", "bf16", 300), ("int4", "fp16", 96), ("nvfp4", "bf16", 3)])
+def test_lora_appended_layer(gpu, fmt, dtype, M):
+    """A layer with a LoRA adapter appended by svdq_append_lora (no
+    re-quantisation) against the oracle's appended layer."""
+    from oracle import svdquant as sq
+    wl = synth.custom_workload(M, 1024, 512, 32, fmt, dtype, n_out=4, factor=40.0, seed=61)
+    pp = G.prepare(wl)
+    A, B = synth.make_lora(3, wl.K, wl.N, 32)
+    q, blob2 = sv.append_lora(pp.p, pp.blob, A, B)
+    pp2 = G.Prepared(wl, q, blob2, pp.sigma, sq.append_lora(pp.ref, A, B), pp.x64)
+    G.compare(pp2, wl.X, G.run_gpu(pp2, wl.X))

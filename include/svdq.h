@@ -140,6 +140,22 @@ svdq_status svdq_append_lora(const svdq_params* p, const void* blob_in, size_t b
                              const float* B, int32_t r_lora, svdq_params* p_out, void* blob_out,
                              size_t blob_out_bytes);
 
+/*
+ * Column shard of a prepared layer, for column-parallel use on several GPUs
+ * (one shard per GPU, each writing its own slice of Y): output features
+ * [n0, n1) of the layer, with n0 and n1 multiples of 256, 0 <= n0 < n1 <= N.
+ * The shard keeps lambda, L1 and the tensor scales of the whole layer and
+ * takes the features' rows of L2, of the 4-bit residual and its scales, and
+ * of the bias, so svdq_linear on the shard gives columns [n0, n1) of the full
+ * layer's output (bit for bit when both run the same GEMM schedule, i.e.
+ * outside the few-token K split).  blob_in (blob_in_bytes, checked as by
+ * svdq_blob_check) is read only; blob_out is a host buffer of blob_out_bytes
+ * >= svdq_blob_bytes(p_out); *p_out receives p with N = n1 - n0.  Errors:
+ * SVDQ_ERR_INVALID_ARG (range, sizes), SVDQ_ERR_BLOB (blob_in).
+ */
+svdq_status svdq_shard_columns(const svdq_params* p, const void* blob_in, size_t blob_in_bytes, int32_t n0,
+                               int32_t n1, svdq_params* p_out, void* blob_out, size_t blob_out_bytes);
+
 /* Device workspace bytes svdq_linear needs for M tokens. */
 size_t svdq_workspace_bytes(const svdq_params* p, int64_t M);
 

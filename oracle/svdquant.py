@@ -167,6 +167,16 @@ def append_lora(p: Prepared, A: np.ndarray, B: np.ndarray) -> Prepared:
                     p.s_gx, p.bias)
 
 
+def shard_columns(p: Prepared, n0: int, n1: int) -> Prepared:
+    """Output features [n0, n1) of a prepared layer: the columns of L2, R, the
+    weight codes and scales and the bias; lambda, L1 and the tensor scales are
+    the whole layer's.  Every output column of the layer depends only on its
+    own weight row, so the shard computes exactly those columns."""
+    wq = WeightQ(p.wq.fmt, p.wq.codes[n0:n1], p.wq.scales[n0:n1], p.wq.s_g)
+    return Prepared(p.fmt, p.dtype, p.rank, p.inv_lambda, p.lam_eff, p.L1, p.L2[:, n0:n1], p.sigma,
+                    p.R[:, n0:n1], wq, p.s_gx, p.bias[n0:n1])
+
+
 # ----------------------------------------------------------------- online side
 def smooth_act(x: np.ndarray, inv_lambda: np.ndarray) -> np.ndarray:
     """X^ = fp32(x) * inv_lambda, one fp32 multiply per element."""

@@ -53,6 +53,7 @@ def _load():
         "svdq_blob_check": (ctypes.c_int, [P, vp, sz]),
         "svdq_blob_export": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
         "svdq_append_lora": (ctypes.c_int, [P, vp, sz, vp, vp, ctypes.c_int32, P, vp, sz]),
+        "svdq_shard_columns": (ctypes.c_int, [P, vp, sz, ctypes.c_int32, ctypes.c_int32, P, vp, sz]),
         "svdq_workspace_bytes": (sz, [P, i64]),
         "svdq_linear": (ctypes.c_int, [P, vp, vp, i64, vp, vp, sz, vp]),
         "svdq_quantize_act": (ctypes.c_int, [P, vp, vp, i64, vp, sz, vp]),
@@ -74,7 +75,7 @@ def _load():
 
 
 _lib = _load()
-EXPORTED = ("svdq_blob_bytes", "svdq_prepare", "svdq_blob_check", "svdq_blob_export", "svdq_append_lora",
+EXPORTED = ("svdq_blob_bytes", "svdq_prepare", "svdq_blob_check", "svdq_blob_export", "svdq_append_lora", "svdq_shard_columns",
             "svdq_workspace_bytes", "svdq_linear", "svdq_quantize_act", "svdq_gemm", "svdq_export_act", "svdq_get_status",
             "svdq_status_string", "svdq_last_error_string", "svdq_probe_cvt", "svdq_probe_div", "svdq_probe_tc",
             "svdq_linear_noalloc", "svdq_probe_timeout")
@@ -162,6 +163,17 @@ def append_lora(p: svdq_params, blob: np.ndarray, A: np.ndarray, B: np.ndarray):
     p_out = svdq_params()
     _check(_lib.svdq_append_lora(ctypes.byref(p), _ptr(blob), blob.nbytes, _ptr(A), _ptr(B), r_lora,
                                  ctypes.byref(p_out), _ptr(out), out.nbytes), "svdq_append_lora")
+    return p_out, out
+
+
+def shard_columns(p: svdq_params, blob: np.ndarray, n0: int, n1: int):
+    """Output features [n0, n1) of a prepared layer as a layer of its own;
+    returns (params with N = n1 - n0, blob)."""
+    q = svdq_params(p.K, n1 - n0, p.rank, p.fmt, p.act_dtype, p.smooth, p.alpha, 0)
+    out = np.zeros(max(blob_bytes(q), 1), np.uint8)
+    p_out = svdq_params()
+    _check(_lib.svdq_shard_columns(ctypes.byref(p), _ptr(blob), blob.nbytes, n0, n1, ctypes.byref(p_out),
+                                   _ptr(out), out.nbytes), "svdq_shard_columns")
     return p_out, out
 
 

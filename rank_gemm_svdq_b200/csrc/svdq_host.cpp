@@ -644,6 +644,43 @@ svdq_status svdq_blob_export(const svdq_params* p, const void* blob, float* inv_
   return SVDQ_OK;
 }
 
+svdq_status svdq_shard_columns(const svdq_params* p, const void* blob_in, size_t blob_in_bytes, int32_t n0,
+                               int32_t n1, svdq_params* p_out, void* blob_out, size_t blob_out_bytes) {
+  svdq_status st = svdq_blob_check(p, blob_in, blob_in_bytes);
+  if (st != SVDQ_OK) return st;
+  if (!p_out || !blob_out || n0 < 0 || n1 > p->N || n0 >= n1 || n0 % 256 != 0 || n1 % 256 != 0)
+    return SVDQ_ERR_INVALID_ARG;
+  svdq_params q = *p;
+  q.N = n1 - n0;
+  const BlobLayout Li = blob_layout(*p), Lo = blob_layout(q);
+  if (blob_out_bytes < Lo.total) return SVDQ_ERR_INVALID_ARG;
+  const int K = p->K, N = p->N, Ns = q.N;
+  const uint8_t* in = (const uint8_t*)blob_in;
+  uint8_t* out = (uint8_t*)blob_out;
+  memset(out, 0, Lo.total);
+  memcpy(out, in, sizeof(BlobHeader));   // tensor scales s_gX, s_gW stay those of the whole layer
+  memcpy(out + Lo.off_inv_lambda, in + Li.off_inv_lambda, (size_t)K * 4);
+  memcpy(out + Lo.off_l1t, in + Li.off_l1t, (size_t)p->rank * K * 2);
+  // every per-column array is ordered by output feature first, so a column
+  // range [n0, n1) (whole 256-column tiles) is one contiguous run of each
+  const size_t w2 = (size_t)lr_width(*p);
+  memcpy(out + Lo.off_l2x, in + Li.off_l2x + (size_t)n0 * w2 * 2, (size_t)Ns * w2 * 2);
+  if (p->fmt == SVDQ_NVFP4) {
+    const size_t tile_row = (size_t)(K / 256) * kWTile;   // one 128-row block over all K slabs
+    memcpy(out + Lo.off_wq, in + Li.off_wq + (size_t)(n0 / 128) * tile_row, (size_t)(Ns / 128) * tile_row);
+  } else {
+    memcpy(out + Lo.off_wq, in + Li.off_wq + (size_t)n0 * K, (size_t)Ns * K);
+    // blocked scales [K/128][N/128][2][128]: one run per 128-wide K slab
+    for (int kt = 0; kt < K / 128; ++kt)
+      memcpy(out + Lo.off_ws + (size_t)kt * (Ns / 128) * 1024,
+             in + Li.off_ws + ((size_t)kt * (N / 128) + n0 / 128) * 1024, (size_t)(Ns / 128) * 1024);
+  }
+  memcpy(out + Lo.off_bias, in + Li.off_bias + (size_t)n0 * 4, (size_t)Ns * 4);
+  finish_header(&q, Lo, out);
+  *p_out = q;
+  return SVDQ_OK;
+}
+
 svdq_status svdq_append_lora(const svdq_params* p, const void* blob_in, size_t blob_in_bytes, const float* A,
                              const float* B, int32_t r_lora, svdq_params* p_out, void* blob_out,
                              size_t blob_out_bytes) {

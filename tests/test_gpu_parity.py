@@ -226,3 +226,22 @@ def test_lora_appended_layer(gpu, fmt, dtype, M):
     q, blob2 = sv.append_lora(pp.p, pp.blob, A, B)
     pp2 = G.Prepared(wl, q, blob2, pp.sigma, sq.append_lora(pp.ref, A, B), pp.x64)
     G.compare(pp2, wl.X, G.run_gpu(pp2, wl.X))
+
+
+@pytest.mark.parametrize("fmt,dtype", [("nvfp4", "bf16"), ("int4", "fp16")])
+def test_column_shards_reassemble_the_layer(gpu, fmt, dtype):
+    """Column shards (one per GPU in column-parallel use) each match the
+    oracle's shard, and side by side they are the full layer's output, bit
+    for bit (same tiles, same K order)."""
+    from oracle import svdquant as sq
+    wl = synth.custom_workload(300, 1024, 1024, 32, fmt, dtype, n_out=4, factor=40.0, seed=71)
+    pp = G.prepare(wl)
+    full = G.run_gpu(pp, wl.X)
+    parts = []
+    for n0, n1 in ((0, 256), (256, 768), (768, 1024)):
+        q, b = sv.shard_columns(pp.p, pp.blob, n0, n1)
+        pps = G.Prepared(wl, q, b, pp.sigma, sq.shard_columns(pp.ref, n0, n1), pp.x64)
+        run = G.run_gpu(pps, wl.X)
+        G.compare(pps, wl.X, run)
+        parts.append(run.Y)
+    assert np.array_equal(np.hstack(parts), full.Y)

@@ -21,6 +21,8 @@ Modules:
   quant      INT4 group-64 and NVFP4 quantisers (fp32 arithmetic)
   svd        one-sided Jacobi SVD in float64 (plain C helper, _jacobi.c)
   svdquant   smoothing, truncated factors, residual, Y
+  kvcache    asymmetric per-channel INT8 KV-cache codec ("VAR-Compressor…",
+             INT8 KV缓存量化)
 
 Pins: tests/test_oracle_*.py check every function against what the pages and
 the mathematics fix (closed forms, invariants, brute force, format tables).

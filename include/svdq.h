@@ -156,6 +156,41 @@ svdq_status svdq_append_lora(const svdq_params* p, const void* blob_in, size_t b
 svdq_status svdq_shard_columns(const svdq_params* p, const void* blob_in, size_t blob_in_bytes, int32_t n0,
                                int32_t n1, svdq_params* p_out, void* blob_out, size_t blob_out_bytes);
 
+/* ------------------------------------------------- INT8 KV-cache codec
+ * Asymmetric per-channel INT8 for a block of cached keys or values
+ * ("VAR-Compressor：在边缘GPU上实现80亿参数视觉自回归模型的高效量化部署",
+ * INT8 KV缓存量化 and KV缓存特性研究: the cache's variance is driven by channels
+ * and its distribution is skewed, so each channel gets its own scale and a
+ * non-centred zero point).  For a block X of T tokens x C channels
+ * (row-major, act dtype), per channel c, in fp32 with round to nearest even:
+ *   lo = min(0, min_t X[t,c]), hi = max(0, max_t X[t,c]),
+ *   scale = (hi - lo) / 255 (1 when hi == lo), zero = clamp(rint(-lo/scale), 0, 255),
+ *   code  = clamp(rint(X/scale) + zero, 0, 255)        (uint8)
+ * and decoding gives (code - zero) * scale rounded to the dtype.  A zero
+ * entry decodes to exactly 0.
+ */
+
+/* Device workspace bytes of svdq_kv_encode for a T x C block (0 if invalid). */
+size_t svdq_kv_workspace_bytes(int64_t T, int32_t C);
+
+/*
+ * Encode a device block.  X: T x C, dtype an svdq_dtype value (SVDQ_BF16 /
+ * SVDQ_F16).  codes: T x C uint8; scale: C fp32; zero: C uint8; workspace:
+ * ws_bytes >= svdq_kv_workspace_bytes(T, C).  All device pointers, 16-byte
+ * aligned, owned by the caller.  T >= 1, C % 256 == 0.  Asynchronous on
+ * `stream` (two kernels).  Errors: SVDQ_ERR_INVALID_ARG, SVDQ_ERR_WORKSPACE,
+ * SVDQ_ERR_ALIGNMENT, SVDQ_ERR_UNSUPPORTED (no sm_100 device), SVDQ_ERR_CUDA.
+ */
+svdq_status svdq_kv_encode(const void* X, int64_t T, int32_t C, int32_t dtype, uint8_t* codes, float* scale,
+                           uint8_t* zero, void* workspace, size_t ws_bytes, svdq_stream stream);
+
+/*
+ * Decode a device block back to dtype: Y[t,c] = dtype((codes[t,c] - zero[c]) * scale[c]).
+ * T >= 1, C % 8 == 0; device pointers 16-byte aligned; asynchronous.
+ */
+svdq_status svdq_kv_decode(const uint8_t* codes, const float* scale, const uint8_t* zero, int64_t T, int32_t C,
+                           int32_t dtype, void* Y, svdq_stream stream);
+
 /* Device workspace bytes svdq_linear needs for M tokens. */
 size_t svdq_workspace_bytes(const svdq_params* p, int64_t M);
 

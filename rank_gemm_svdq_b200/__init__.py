@@ -54,6 +54,9 @@ def _load():
         "svdq_blob_export": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
         "svdq_append_lora": (ctypes.c_int, [P, vp, sz, vp, vp, ctypes.c_int32, P, vp, sz]),
         "svdq_shard_columns": (ctypes.c_int, [P, vp, sz, ctypes.c_int32, ctypes.c_int32, P, vp, sz]),
+        "svdq_kv_workspace_bytes": (sz, [i64, ctypes.c_int32]),
+        "svdq_kv_encode": (ctypes.c_int, [vp, i64, ctypes.c_int32, ctypes.c_int32, vp, vp, vp, vp, sz, vp]),
+        "svdq_kv_decode": (ctypes.c_int, [vp, vp, vp, i64, ctypes.c_int32, ctypes.c_int32, vp, vp]),
         "svdq_workspace_bytes": (sz, [P, i64]),
         "svdq_linear": (ctypes.c_int, [P, vp, vp, i64, vp, vp, sz, vp]),
         "svdq_quantize_act": (ctypes.c_int, [P, vp, vp, i64, vp, sz, vp]),
@@ -78,7 +81,8 @@ _lib = _load()
 EXPORTED = ("svdq_blob_bytes", "svdq_prepare", "svdq_blob_check", "svdq_blob_export", "svdq_append_lora", "svdq_shard_columns",
             "svdq_workspace_bytes", "svdq_linear", "svdq_quantize_act", "svdq_gemm", "svdq_export_act", "svdq_get_status",
             "svdq_status_string", "svdq_last_error_string", "svdq_probe_cvt", "svdq_probe_div", "svdq_probe_tc",
-            "svdq_linear_noalloc", "svdq_probe_timeout")
+            "svdq_linear_noalloc", "svdq_probe_timeout", "svdq_kv_workspace_bytes", "svdq_kv_encode",
+            "svdq_kv_decode")
 NOALLOC_SCRATCH_BYTES = 16 << 20   # SVDQ_NOALLOC_SCRATCH_BYTES
 
 
@@ -198,6 +202,22 @@ def linear(p: svdq_params, blob_dev, X, M: int, Y, workspace, stream=None):
     st = _lib.svdq_linear(ctypes.byref(p), _ptr(blob_dev), _ptr(X), M, _ptr(Y), _ptr(workspace),
                           workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "svdq_linear")
+
+
+def kv_workspace_bytes(T: int, C: int) -> int:
+    return _lib.svdq_kv_workspace_bytes(T, C)
+
+
+def kv_encode(X, T: int, C: int, dtype: str, codes, scale, zero, workspace, stream=None):
+    """Asymmetric per-channel INT8 encode of a T x C cache block (device tensors)."""
+    st = _lib.svdq_kv_encode(_ptr(X), T, C, DTYPE[dtype], _ptr(codes), _ptr(scale), _ptr(zero), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "svdq_kv_encode")
+
+
+def kv_decode(codes, scale, zero, T: int, C: int, dtype: str, Y, stream=None):
+    st = _lib.svdq_kv_decode(_ptr(codes), _ptr(scale), _ptr(zero), T, C, DTYPE[dtype], _ptr(Y), _stream(stream))
+    _check(st, "svdq_kv_decode")
 
 
 def linear_noalloc(p: svdq_params, blob_dev, X, M: int, Y, stream=None):

@@ -13,7 +13,7 @@ BUILD = os.path.join(HERE, "_build")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
-SOURCES_CU = ["svdq_device.cu"]
+SOURCES_CU = ["svdq_device.cu", "kv_device.cu"]
 SOURCES_CPP = ["svdq_host.cpp"]
 HEADERS = ["layout.h", "ptx.cuh"]
 

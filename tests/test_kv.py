@@ -70,3 +70,60 @@ def test_asymmetric_beats_symmetric_on_skewed_data():
     assert np.all(s <= sym * (1 + 1e-6))
     assert np.mean(np.abs(kv.decode(q, s, z) - x)) < 0.75 * np.mean(
         np.abs(np.clip(np.rint(x / sym), -127, 127) * sym - x))
+
+
+def _block_bits(T, C, dtype, seed):
+    """A skewed T x C block as dtype bit patterns (uint16) and its float64 values."""
+    g = synth.normal(seed, "X", T * C).reshape(T, C)
+    scale = np.exp(synth.normal(seed, "extra", C) * 1.2)
+    x = (np.exp(0.6 * g) - 1.2) * scale[None, :]
+    x[:, :3] = 0.0                                   # all-zero channels (scale 1, zero point 0)
+    bits = synth.to_dtype(x, dtype)
+    bits = bits.view(np.uint16) if dtype == "fp16" else bits
+    return bits, synth.dtype_to_f64(synth.to_dtype(x, dtype), dtype)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("T,C,dtype", [(1, 256, "bf16"), (300, 512, "fp16"), (257, 768, "bf16"),
+                                       (4096, 4096, "bf16")])
+def test_gpu_kv_codec_matches_oracle(gpu, T, C, dtype):
+    """svdq_kv_encode / svdq_kv_decode against the oracle: codes, scales and
+    zero points bit-exact, decoded values bit-exact after rounding to the dtype.
+    The largest case (a 4096-token x 4096-channel VAR-like block) is also timed."""
+    import torch
+    import rank_gemm_svdq_b200 as sv
+    bits, x = _block_bits(T, C, dtype, seed=T + C)
+    X = torch.from_numpy(bits.view(np.int16)).cuda()
+    codes = torch.empty((T, C), dtype=torch.uint8, device="cuda")
+    scale = torch.empty(C, dtype=torch.float32, device="cuda")
+    zero = torch.empty(C, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(sv.kv_workspace_bytes(T, C), dtype=torch.uint8, device="cuda")
+    sv.kv_encode(X, T, C, dtype, codes, scale, zero, ws)
+    Y = torch.empty((T, C), dtype=torch.int16, device="cuda")
+    sv.kv_decode(codes, scale, zero, T, C, dtype, Y)
+    torch.cuda.synchronize()
+    q, s, z = kv.encode(x)
+    assert np.array_equal(scale.cpu().numpy().view(np.uint32), s.view(np.uint32))
+    assert np.array_equal(zero.cpu().numpy(), z)
+    assert np.array_equal(codes.cpu().numpy(), q)
+    ref = synth.to_dtype(kv.decode(q, s, z), dtype)
+    ref = ref.view(np.uint16) if dtype == "fp16" else ref
+    assert np.array_equal(Y.cpu().numpy().view(np.uint16), ref)
+    if T * C >= 1 << 24:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+        def timed(fn):
+            ts = []
+            for i in range(12):
+                flush.fill_(i)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(); fn(); b.record()
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b) * 1e3)
+            return float(np.median(ts[2:]))
+        te = timed(lambda: sv.kv_encode(X, T, C, dtype, codes, scale, zero, ws))
+        td = timed(lambda: sv.kv_decode(codes, scale, zero, T, C, dtype, Y))
+        enc_bytes = T * C * 2 + T * C + C * 5          # X in, codes + scales + zero points out
+        dec_bytes = T * C + C * 5 + T * C * 2
+        print(f"kv {T}x{C} {dtype}: encode {te:.1f} us = {enc_bytes / te / 1e3:.0f} GB/s, "
+              f"decode {td:.1f} us = {dec_bytes / td / 1e3:.0f} GB/s (algorithmic bytes)")

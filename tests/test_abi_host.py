@@ -139,3 +139,24 @@ def test_zero_weight_and_zero_calibration():
     c = sv.blob_export(p, blob)
     assert np.all(c.inv_lambda == 1.0) and np.all(c.wcodes == 0) and np.all(c.bias == 0)
     assert c.s_gx == 1.0 and c.s_gw == 1.0 and np.all(sigma == 0)
+
+
+def test_kv_codec_argument_checks_need_no_gpu():
+    """svdq_kv_encode / svdq_kv_decode reject bad shapes, dtypes, workspaces
+    and misaligned pointers before touching a device (the pointers below are
+    never dereferenced)."""
+    L = sv.lib()
+    A = 1 << 20                                # a 16-byte aligned fake address
+    assert L.svdq_kv_workspace_bytes(0, 256) == 0
+    assert L.svdq_kv_workspace_bytes(257, 512) == 2 * 2 * 512 * 4
+    ws = L.svdq_kv_workspace_bytes(300, 512)
+    enc = lambda X, T, C, dt, q, s, z, w, wb: L.svdq_kv_encode(X, T, C, dt, q, s, z, w, wb, None)
+    assert enc(A, 0, 512, sv.BF16, A, A, A, A, ws) == sv.ERR_INVALID_ARG        # no tokens
+    assert enc(A, 300, 320, sv.BF16, A, A, A, A, ws) == sv.ERR_INVALID_ARG      # C % 256
+    assert enc(A, 300, 512, 9, A, A, A, A, ws) == sv.ERR_INVALID_ARG            # dtype
+    assert enc(None, 300, 512, sv.BF16, A, A, A, A, ws) == sv.ERR_INVALID_ARG   # null
+    assert enc(A, 300, 512, sv.BF16, A, A, A, A, ws - 1) == sv.ERR_WORKSPACE
+    assert enc(A + 2, 300, 512, sv.BF16, A, A, A, A, ws) == sv.ERR_ALIGNMENT
+    dec = lambda q, s, z, T, C, dt, Y: L.svdq_kv_decode(q, s, z, T, C, dt, Y, None)
+    assert dec(A, A, A, 10, 12, sv.BF16, A) == sv.ERR_INVALID_ARG               # C % 8
+    assert dec(A, A, A, 10, 64, sv.F16, A + 8) == sv.ERR_ALIGNMENT

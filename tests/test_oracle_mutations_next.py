@@ -1,0 +1,107 @@
+"""Planted mistakes in the oracle's next-row functions (KV-cache codec, LoRA
+append, column shards) must each fail at least one of their pins (the CPU
+tests of tests/test_kv.py, tests/test_lora.py and tests/test_shard.py)."""
+import numpy as np
+import pytest
+
+import oracle.formats as formats
+import oracle.kvcache as kv
+import oracle.svdquant as sq
+from tests import test_kv as TK
+from tests import test_lora as TL
+from tests import test_shard as TS
+
+F32 = np.float32
+
+
+def _run(pins):
+    failures = 0
+    for pin in pins:
+        try:
+            pin()
+        except Exception:
+            failures += 1
+    return failures
+
+
+KV_PINS = [TK.test_golden_codes, TK.test_round_trip_error_is_half_a_step, TK.test_range_ends_map_to_the_code_ends,
+           TK.test_asymmetric_beats_symmetric_on_skewed_data]
+LORA_PINS = [lambda: TL.test_oracle_lora_adds_exactly_xab_without_smoothing("nvfp4"),
+             lambda: TL.test_oracle_lora_with_smoothing_matches_xab_to_the_dtype("int4", "fp16")]
+SHARD_PINS = [lambda: TS.test_oracle_shard_is_the_full_layers_columns("int4", "fp16"),
+              lambda: TS.test_oracle_shard_is_the_full_layers_columns("nvfp4", "bf16")]
+
+
+def _params(divisor=255.0, widen=True, zsign=-1.0):
+    def channel_params(x):
+        x32 = np.asarray(x, dtype=np.float64).astype(F32)
+        lo, hi = x32.min(axis=0), x32.max(axis=0)
+        if widen:
+            lo, hi = np.minimum(lo, F32(0)), np.maximum(hi, F32(0))
+        s = ((hi - lo) / F32(divisor)).astype(F32)
+        s = np.where(s == 0, F32(1.0), s).astype(F32)
+        z = np.clip(np.rint((F32(zsign) * lo) / s), 0, 255).astype(np.uint8)
+        return s, z
+    return channel_params
+
+
+def _encode_ties_up(x):
+    s, z = kv.channel_params(x)
+    x32 = np.asarray(x, dtype=np.float64).astype(F32)
+    q = np.floor(x32 / s[None, :] + 0.5).astype(np.float64) + z[None, :]
+    return np.clip(q, 0, 255).astype(np.uint8), s, z
+
+
+def _decode_plus_zero(q, s, z):
+    d = (q.astype(np.int32) + z[None, :].astype(np.int32)).astype(F32)
+    return (d * s[None, :]).astype(F32).astype(np.float64)
+
+
+def _lora_without_lambda(p, A, B):
+    A = np.asarray(A, dtype=np.float64); B = np.asarray(B, dtype=np.float64)
+    return sq.Prepared(p.fmt, p.dtype, p.rank + A.shape[1], p.inv_lambda, p.lam_eff,
+                       np.hstack([p.L1, formats.to_dtype(A, p.dtype)]), np.vstack([p.L2, formats.to_dtype(B, p.dtype)]),
+                       p.sigma, p.R, p.wq, p.s_gx, p.bias)
+
+
+def _lora_lambda_divides(p, A, B):
+    A = np.asarray(A, dtype=np.float64); B = np.asarray(B, dtype=np.float64)
+    return sq.Prepared(p.fmt, p.dtype, p.rank + A.shape[1], p.inv_lambda, p.lam_eff,
+                       np.hstack([p.L1, formats.to_dtype(A / p.lam_eff[:, None], p.dtype)]),
+                       np.vstack([p.L2, formats.to_dtype(B, p.dtype)]), p.sigma, p.R, p.wq, p.s_gx, p.bias)
+
+
+def _shard_bias_unshifted(p, n0, n1):
+    wq = sq.WeightQ(p.wq.fmt, p.wq.codes[n0:n1], p.wq.scales[n0:n1], p.wq.s_g)
+    return sq.Prepared(p.fmt, p.dtype, p.rank, p.inv_lambda, p.lam_eff, p.L1, p.L2[:, n0:n1], p.sigma,
+                       p.R[:, n0:n1], wq, p.s_gx, p.bias[:n1 - n0])
+
+
+def _shard_l2_unshifted(p, n0, n1):
+    wq = sq.WeightQ(p.wq.fmt, p.wq.codes[n0:n1], p.wq.scales[n0:n1], p.wq.s_g)
+    return sq.Prepared(p.fmt, p.dtype, p.rank, p.inv_lambda, p.lam_eff, p.L1, p.L2[:, :n1 - n0], p.sigma,
+                       p.R[:, n0:n1], wq, p.s_gx, p.bias[n0:n1])
+
+
+MUTATIONS = {
+    "kv_divisor_256": (kv, "channel_params", _params(divisor=256.0), KV_PINS),
+    "kv_zero_point_sign": (kv, "channel_params", _params(zsign=1.0), KV_PINS),
+    "kv_range_not_widened": (kv, "channel_params", _params(widen=False), KV_PINS),
+    "kv_ties_up": (kv, "encode", _encode_ties_up, KV_PINS),
+    "kv_decode_adds_zero": (kv, "decode", _decode_plus_zero, KV_PINS),
+    "lora_lambda_dropped": (sq, "append_lora", _lora_without_lambda, LORA_PINS),
+    "lora_lambda_divides": (sq, "append_lora", _lora_lambda_divides, LORA_PINS),
+    "shard_bias_unshifted": (sq, "shard_columns", _shard_bias_unshifted, SHARD_PINS),
+    "shard_l2_unshifted": (sq, "shard_columns", _shard_l2_unshifted, SHARD_PINS),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    mod, attr, fn, pins = MUTATIONS[name]
+    monkeypatch.setattr(mod, attr, fn)
+    assert _run(pins) > 0, f"no pin caught the planted mistake {name!r}"
+
+
+def test_unmutated_pins_pass():
+    assert _run(KV_PINS + LORA_PINS + SHARD_PINS) == 0

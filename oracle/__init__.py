@@ -25,7 +25,12 @@ Modules:
              INT8 KV缓存量化)
 
 Pins: tests/test_oracle_*.py check every function against what the pages and
-the mathematics fix (closed forms, invariants, brute force, format tables).
+the mathematics fix (closed forms, invariants, brute force, format tables);
+tests/test_kv.py (a hand-worked fixture and the codec's invariants),
+tests/test_lora.py (the appended layer against plain X A B products) and
+tests/test_shard.py (a shard against the full layer's columns) pin the
+next-row functions, and tests/test_oracle_mutations*.py plant mistakes that
+the pins must catch.
 Functions whose result is not pinned say "parity unpinned" in their docstring;
 there are none at present.
 """

@@ -22,6 +22,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/svdq.h"
 
 namespace svdq {
@@ -173,15 +175,18 @@ __global__ void __launch_bounds__(256) kv_decode_kernel(const uint8_t* __restric
 
 // sm_100 check, cached per device (cudaGetDeviceProperties costs milliseconds)
 bool device_ok() {
-  static int state[64] = {};   // 0 unknown, 1 ok, 2 not ok
+  static std::atomic<int> state[64];   // 0 unknown, 1 ok, 2 not ok (zero-initialised)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
-  if (dev < 64 && state[dev]) return state[dev] == 1;
+  if (dev < 64) {
+    const int known = state[dev].load(std::memory_order_relaxed);
+    if (known) return known == 1;
+  }
   int major = 0, minor = 0;
   const bool ok = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
                   cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
                   major == 10 && minor == 0;
-  if (dev < 64) state[dev] = ok ? 1 : 2;
+  if (dev < 64) state[dev].store(ok ? 1 : 2, std::memory_order_relaxed);
   return ok;
 }
 

@@ -181,6 +181,35 @@ def shard_columns(p: svdq_params, blob: np.ndarray, n0: int, n1: int):
     return p_out, out
 
 
+def shard_bounds(N: int, world: int) -> list[tuple[int, int]]:
+    """Split N output features into `world` column ranges of whole 256-column
+    tiles, as even as possible (the first ranges take the extra tiles)."""
+    tiles = N // 256
+    assert N % 256 == 0 and 1 <= world <= tiles, (N, world)
+    base, extra = divmod(tiles, world)
+    out, n0 = [], 0
+    for r in range(world):
+        n1 = n0 + 256 * (base + (1 if r < extra else 0))
+        out.append((n0, n1))
+        n0 = n1
+    return out
+
+
+def all_gather_columns(y_local, bounds, group=None):
+    """Column-parallel output: every rank holds Y[:, n0:n1] of its own range;
+    returns the whole Y (M x N) on every rank (torch.distributed all_gather,
+    NCCL between GPUs).  Ranges may differ in width by one tile."""
+    import torch
+    import torch.distributed as dist
+    M = y_local.shape[0]
+    width = max(n1 - n0 for n0, n1 in bounds)
+    pad = torch.zeros((M, width), dtype=y_local.dtype, device=y_local.device)
+    pad[:, :y_local.shape[1]] = y_local
+    parts = [torch.empty_like(pad) for _ in bounds]
+    dist.all_gather(parts, pad.contiguous(), group=group)
+    return torch.cat([t[:, :n1 - n0] for t, (n0, n1) in zip(parts, bounds)], dim=1)
+
+
 def blob_export(p: svdq_params, blob: np.ndarray) -> BlobContents:
     K, N, r = p.K, p.N, p.rank
     inv = np.zeros(K, np.float32)

@@ -404,3 +404,68 @@ def pin_low_rank_helps(sq):
         e0 = sq.rel_fro(sq.forward(x, sq.prepare(x, Wt, b, 0, fmt, "fp16", smooth=False)), ref)
         er = sq.rel_fro(sq.forward(x, sq.prepare(x, Wt, b, 16, fmt, "fp16")), ref)
         assert er < e0, (fmt, er, e0)
+
+
+# ------------------------------------------------------------------ activation side
+def _golden_lines(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                yield [part.strip() for part in line.split("|")]
+
+
+def pin_act_tensor_scale_golden(sq):
+    """The static NVFP4 activation tensor scale is amax of the SMOOTHED
+    calibration activations over 2688, bit for bit on hand-worked cases
+    (golden file: the amax of X and of X^ sit in different places)."""
+    for rows, inv, bits in _golden_lines("act_tensor_scale.txt"):
+        x_cal = np.array([[float(t) for t in r.split()] for r in rows.split(";")])
+        inv_l = np.array([float(t) for t in inv.split()], dtype=np.float32)
+        s = sq.act_tensor_scale(x_cal, inv_l)
+        assert np.float32(s).view(np.uint32) == np.uint32(int(bits, 16)), (rows, float(s), bits)
+
+
+def _bare_layer(sq, fmt, inv_l, s_gx):
+    """A rank-0 layer holding only what the activation side reads."""
+    K = len(inv_l)
+    return sq.Prepared(fmt, "fp16", 0, inv_l, 1.0 / inv_l.astype(np.float64), np.zeros((K, 0)),
+                       np.zeros((0, 1)), None, None, None, np.float32(s_gx), np.zeros(1, np.float32))
+
+
+def pin_act_codes_golden(sq):
+    """Per-token activation codes and scales of quantize_act are those of
+    X^ = fl32(x) * inv_lambda (hand-worked golden file: ties to even, signed
+    zero, the block scale from the smoothed block amax)."""
+    for fmt, sg, inv, xs, scale, codes in _golden_lines("act_codes_smoothed.txt"):
+        inv_l = np.array([float(t) for t in inv.split()], dtype=np.float32)
+        x = np.array([[float(t) for t in xs.split()]])
+        a = sq.quantize_act(x, _bare_layer(sq, fmt, inv_l, float(sg)), group=64)
+        if fmt == "nvfp4":
+            assert a.scales.ravel().tolist() == [int(t, 16) for t in scale.split()], (a.scales, scale)
+            assert a.codes.ravel().tolist() == [int(t, 16) for t in codes.split()], a.codes
+        else:
+            assert a.scales.ravel().tolist() == [float(t) for t in scale.split()], (a.scales, scale)
+            assert a.codes.ravel().tolist() == [int(t) for t in codes.split()], a.codes
+
+
+def pin_act_scale_in_prepare(sq):
+    """prepare() takes s_gX from the calibration activations after smoothing:
+    recomputed here with plain loops over every element on a layer with
+    outlier channels (where amax(X) and amax(X^) differ by far)."""
+    rng = np.random.default_rng(18)
+    M, K, N = 24, 64, 32
+    x = rng.standard_normal((M, K)); x[:, [4, 33]] *= 60
+    x = x.astype(np.float16).astype(np.float64)
+    Wt = (rng.standard_normal((N, K)) / 8).astype(np.float32)
+    p = sq.prepare(x, Wt, None, 0, "nvfp4", "fp16")
+    amax = 0.0
+    for m in range(M):
+        for j in range(K):
+            v = abs(float(np.float32(np.float32(x[m, j]) * p.inv_lambda[j])))
+            amax = v if v > amax else amax
+    assert amax < 0.5 * float(np.abs(x).max())        # the smoothing really moved the range
+    expect = Fraction(amax) / 2688
+    got = Fraction(float(p.s_gx))
+    # fl32 of the exact quotient: within half an fp32 ulp of it
+    ulp = Fraction(2) ** (math.frexp(float(expect))[1] - 24)
+    assert abs(got - expect) <= ulp / 2, (float(got), float(expect))

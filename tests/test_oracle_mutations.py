@@ -30,6 +30,10 @@ def _run_all_pins():
         lambda: P.pin_bruteforce_nvfp4(sq),
         lambda: P.pin_special_cases(sq),
         lambda: P.pin_on_grid_lossless(sq),
+        lambda: P.pin_low_rank_helps(sq),
+        lambda: P.pin_act_tensor_scale_golden(sq),
+        lambda: P.pin_act_codes_golden(sq),
+        lambda: P.pin_act_scale_in_prepare(sq),
     ]
     failures = 0
     for pin in pins:
@@ -120,6 +124,25 @@ def _to_dtype_truncate(x, dtype):
     return np.ldexp(np.trunc(np.ldexp(m, bits)), e - bits)
 
 
+def _act_tensor_scale_unsmoothed(x_cal, inv_lambda):
+    x = np.asarray(x_cal, dtype=np.float64).astype(F32)
+    return quant.nvfp4_tensor_scale(np.abs(x).max() if x.size else 0.0)
+
+
+def _quantize_act_codes_unsmoothed(x, p, group=64):
+    a = _orig_qa(x, p, group)
+    x32 = np.asarray(x, dtype=np.float64).astype(F32)
+    if p.fmt == "int4":
+        a.codes, a.scales = quant.int4_group_quant(x32, group)
+    else:
+        a.codes, a.scales = quant.nvfp4_quant(x32, p.s_gx)
+    return a
+
+
+def _smooth_act_divides(x, inv_lambda):
+    return (np.asarray(x, dtype=np.float64).astype(F32) / np.asarray(inv_lambda, dtype=F32)).astype(F32)
+
+
 MUTATIONS = {
     "residual_sign": (sq, "residual", _residual_plus),
     "smoothing_direction": (sq, "smooth_weight", _smooth_weight_divides),
@@ -130,6 +153,9 @@ MUTATIONS = {
     "group_scale_index": (sq, "main_product", _main_product_swapped_group),
     "e2m1_ties_up": (formats, "e2m1_encode", _e2m1_tie_up),
     "dtype_rounding_truncates": (formats, "to_dtype", _to_dtype_truncate),
+    "act_tensor_scale_from_unsmoothed_x": (sq, "act_tensor_scale", _act_tensor_scale_unsmoothed),
+    "act_codes_from_unsmoothed_x": (sq, "quantize_act", _quantize_act_codes_unsmoothed),
+    "act_smoothing_divides": (sq, "smooth_act", _smooth_act_divides),
 }
 
 

@@ -71,3 +71,15 @@ def test_on_grid_lossless():
 
 def test_low_rank_branch_lowers_error():
     P.pin_low_rank_helps(svdquant)
+
+
+def test_act_tensor_scale_golden():
+    P.pin_act_tensor_scale_golden(svdquant)
+
+
+def test_act_codes_from_smoothed_x_golden():
+    P.pin_act_codes_golden(svdquant)
+
+
+def test_act_tensor_scale_in_prepare():
+    P.pin_act_scale_in_prepare(svdquant)

@@ -272,19 +272,15 @@ svdq_status svdq_probe_div(const float* v, const float* d, int64_t n, float* q, 
 svdq_status svdq_probe_timeout(int64_t limit_ns, svdq_stream stream);
 
 /*
- * Measurement hook: tensor-core operation rate.  Launches `ctas` CTAs (pairs
- * of CTAs for op 1); in each, one thread issues `iters` back-to-back tcgen05
- * operations of kind `op` on zeroed shared memory and writes the clock64
- * cycles it took (issue to completion) to cycles[cta] (device, ctas entries).
+ * Measurement hook: tensor-core MMA rate, the denominators of the GEMM
+ * rooflines.  Launches `ctas` CTAs (rounded up to whole CTA pairs for op 1);
+ * in each, one thread issues `iters` (1 .. 2^24) back-to-back tcgen05 MMAs of
+ * kind `op` on zeroed shared memory and writes the clock64 cycles it took
+ * (issue to completion) to cycles[cta] (device, one entry per launched CTA).
  *   0 mxf4nvf4 128x256x64   1 mxf4nvf4 256x256x64 (CTA pair)
  *   2 bf16 128x256x16       3 E4M3 128x256x32      4 s8 128x256x32
- *   5 scale-factor copy (tcgen05.cp 32x128b.warpx4) only
- *   6 op 0 + 12 copies (32x128b.warpx4) per 4 MMAs
- *   7 op 0 + 6 copies (128x256b) per 4 MMAs
- *   8 tcgen05.st 32x32b.x32 (+ wait) by 4 warps; cycles[ctas * w + cta], w = 1..4
- *   9 op 0 while 4 other warps store 48 TMEM columns per 4 MMAs (warp cycles as op 8)
- *   10 op 1 + 12 copies (cta_group::2 32x128b.warpx4) per 4 MMAs (CTA pair)
- * cycles must hold 5 * ctas entries.  Time the launch with events on `stream` to get the chip-wide rate.
+ * Time the launch with events on `stream` for the chip-wide rate
+ * (2 M N K flops per MMA).  Asynchronous; SVDQ_ERR_INVALID_ARG outside these ranges.
  */
 svdq_status svdq_probe_tc(int op, int iters, int ctas, unsigned long long* cycles, svdq_stream stream);
 
@@ -310,6 +306,9 @@ svdq_status svdq_probe_tc(int op, int iters, int ctas, unsigned long long* cycle
  * The first call on each device performs one-time set-up with that device
  * current (device query, kernel attributes, and the lookup of the scratch
  * buffer's device address); make that first call before any stream capture.
+ * That set-up is kept for the life of the process: after cudaDeviceReset on a
+ * device the kept address and attributes are stale, so do not call the
+ * library on that device again in the same process.
  * There is ONE scratch buffer per device: calls that may overlap on the GPU
  * (different streams, or different host threads, without ordering between
  * them) race on it and corrupt each other's results.  Order such calls.

@@ -71,3 +71,13 @@ def jacobi_svd(A: np.ndarray, tol: float = 1e-15, max_sweeps: int = 60):
     if transpose:                          # A = B^T = V diag(s) U^T
         return np.ascontiguousarray(V), s, np.ascontiguousarray(U.T)
     return np.ascontiguousarray(U), s, np.ascontiguousarray(V.T)
+
+
+def lapack_svd(A: np.ndarray):
+    """Thin SVD of A by LAPACK (numpy.linalg.svd, a library routine), in the
+    same form as jacobi_svd.  For layers too large for the Jacobi sweeps to
+    finish in minutes (the benchmark's reference arm and error report); the
+    two agree on the truncated product L1 L2 up to rounding (pinned)."""
+    A = np.asarray(A, dtype=np.float64)
+    U, s, Vt = np.linalg.svd(A, full_matrices=False)
+    return U, s, Vt

@@ -34,7 +34,7 @@ from dataclasses import dataclass
 import numpy as np
 
 from . import formats, quant
-from .svd import jacobi_svd
+from .svd import jacobi_svd, lapack_svd
 
 F32 = np.float32
 
@@ -65,13 +65,14 @@ def smooth_weight(Wt: np.ndarray, lam_eff: np.ndarray) -> np.ndarray:
     return np.asarray(Wt, dtype=np.float64).T * lam_eff[:, None]
 
 
-def low_rank_factors(W_hat: np.ndarray, rank: int, dtype: str):
+def low_rank_factors(W_hat: np.ndarray, rank: int, dtype: str, svd: str = "jacobi"):
     """Top-`rank` SVD factors of W^, rounded to the 16-bit dtype.
 
     Returns (L1 K x r, L2 r x N, all singular values), factors as float64
-    holding dtype values.
+    holding dtype values.  svd: "jacobi" (the oracle's own sweeps) or
+    "lapack" (numpy's routine, for full-size layers).
     """
-    U, s, Vt = jacobi_svd(W_hat)
+    U, s, Vt = jacobi_svd(W_hat) if svd == "jacobi" else lapack_svd(W_hat)
     L1 = formats.to_dtype(U[:, :rank] * s[None, :rank], dtype)
     L2 = formats.to_dtype(Vt[:rank, :], dtype)
     return L1, L2, s
@@ -129,15 +130,16 @@ def act_tensor_scale(x_cal: np.ndarray, inv_lambda: np.ndarray) -> np.float32:
 
 
 def prepare(x_cal, Wt, bias, rank, fmt, dtype, alpha=0.5, smooth=True, group=64,
-            factors=None) -> Prepared:
+            factors=None, svd="jacobi") -> Prepared:
     """Offline side of the layer.  `factors` = (inv_lambda, L1, L2) replaces the
     oracle's own smoothing/SVD (used to re-derive R and its codes from another
-    implementation's stored factors)."""
+    implementation's stored factors).  `svd` picks the SVD routine (see
+    low_rank_factors)."""
     if factors is None:
         inv_lambda, lam_eff = smoothing_factors(x_cal, Wt, alpha, smooth)
         W_hat = smooth_weight(Wt, lam_eff)
         if rank > 0:
-            L1, L2, sigma = low_rank_factors(W_hat, rank, dtype)
+            L1, L2, sigma = low_rank_factors(W_hat, rank, dtype, svd)
         else:
             L1 = np.zeros((W_hat.shape[0], 0)); L2 = np.zeros((0, W_hat.shape[1])); sigma = None
     else:

@@ -1235,28 +1235,22 @@ __global__ void probe_cvt_kernel(const float* in, int64_t n, uint8_t* e2m1, uint
 
 
 // ------------------------------------------------------------ tensor-core rate probe
-// Measures the issue-limited throughput of tcgen05 operations on this GPU:
-// one thread per CTA issues `iters` operations back to back on zeroed shared
-// memory, then waits (bounded) for their completion.  Used for the roofline
-// denominators (dense FP4 / FP8 / INT8 / BF16 tensor peaks as this part runs
-// them) and to cost the scale-factor copies of the block-scaled GEMM.
+// Measures the issue-limited throughput of tcgen05 MMAs on this GPU: one
+// thread per CTA issues `iters` MMAs back to back on zeroed shared memory,
+// then waits (bounded) for their completion.  These are the tensor peaks the
+// kernels are held against (dense FP4 / FP8 / INT8 / BF16 as this part runs
+// them):
 //   op 0  kind::mxf4nvf4 block16, M=128 N=256 K=64        (1 CTA)
 //   op 1  kind::mxf4nvf4 block16, M=256 N=256 K=64        (CTA pair)
 //   op 2  kind::f16 (bf16),      M=128 N=256 K=16
 //   op 3  kind::f8f6f4 (E4M3),   M=128 N=256 K=32
 //   op 4  kind::i8 (s8),         M=128 N=256 K=32
-//   op 5  tcgen05.cp 32x128b.warpx4 only
-//   op 6  op 0 with 12 scale-factor copies (32x128b.warpx4) per 4 MMAs
-//   op 7  op 0 with 6 scale-factor copies (128x256b) per 4 MMAs
-//   op 8  tcgen05.st 32x32b.x32 + wait::st by 4 warps (one per lane quarter)
-//   op 9  op 0 while 4 other warps store 48 columns (x16 + x32) per 4 MMAs
-//   op 10 op 1 with 12 scale-factor copies (cta_group::2 32x128b.warpx4) per 4 MMAs
 constexpr int kProbeSmem = 16384 + 32768 + 16384 + 1024;
 
 template <bool kPair>
 __device__ __forceinline__ void probe_body(int op, int iters, unsigned long long* cycles) {
   // every tcgen05 instruction of a kernel uses the same cta_group, so the
-  // pair kernel only runs op 1 and the single-CTA kernel every other op
+  // pair kernel only runs op 1 and the single-CTA kernel ops 0 and 2-4
   extern __shared__ __align__(1024) uint8_t psm_raw[];
   __shared__ uint64_t done_bar;
   __shared__ uint32_t tbase_sh;
@@ -1288,8 +1282,6 @@ __device__ __forceinline__ void probe_body(int op, int iters, unsigned long long
     for (int i = 0; i < iters; ++i) {
       const uint32_t acc = i > 0;
       if constexpr (kPair) {
-        if (op == 10 && (i & 3) == 0)
-          for (int q = 0; q < 12; ++q) tmem_cp_32x128b_x4_pair(t + 256 + 4 * q, desc_sf_32x16(sf + 512 * q));
         mma_nvf4_pair(t, desc_k_sw128(a), desc_k_sw128(b), idesc_nvf4(256, 256), t + 256 + 4 * (i & 3),
                       t + 288 + 8 * (i & 3), acc);
       } else {
@@ -1298,22 +1290,6 @@ __device__ __forceinline__ void probe_body(int op, int iters, unsigned long long
           case 2: mma_f16(t, desc_k_sw128(a), desc_k_sw128(b), idesc_f16_bf16(128, 256), acc); break;
           case 3: mma_f8(t, desc_k_sw128(a), desc_k_sw128(b), idesc_f8_e4m3(128, 256), acc); break;
           case 4: mma_i8(t, desc_k_sw128(a), desc_k_sw128(b), idesc_i8(128, 256), acc); break;
-          case 5: tmem_cp_32x128b_x4(t + 256 + 4 * (i & 15), desc_sf_32x16(sf + 512 * (i & 15))); break;
-          case 6:
-            if ((i & 3) == 0)
-              for (int q = 0; q < 12; ++q) tmem_cp_32x128b_x4(t + 256 + 4 * q, desc_sf_32x16(sf + 512 * q));
-            mma_nvf4(t, desc_k_sw128(a), desc_k_sw128(b), idesc_nvf4(128, 256), t + 256 + 4 * (i & 3),
-                     t + 288 + 8 * (i & 3), acc);
-            break;
-          case 7:
-            if ((i & 3) == 0)
-              for (int q = 0; q < 6; ++q) tmem_cp_128x256b(t + 256 + 8 * q, desc_sf_32x16(sf + 2048 * q));
-            mma_nvf4(t, desc_k_sw128(a), desc_k_sw128(b), idesc_nvf4(128, 256), t + 256 + 4 * (i & 3),
-                     t + 288 + 8 * (i & 3), acc);
-            break;
-          case 9:
-            mma_nvf4(t, desc_k_sw128(a), desc_k_sw128(b), idesc_nvf4(128, 256), t + 256, t + 288, acc);
-            break;
           default: break;
         }
       }
@@ -1321,25 +1297,6 @@ __device__ __forceinline__ void probe_body(int op, int iters, unsigned long long
     if constexpr (kPair) mma_commit_pair(&done_bar, 0x3); else mma_commit(&done_bar);
     mbar_wait(&done_bar, 0, &abort_sh);
     cycles[blockIdx.x] = clock64() - t0;
-  }
-  if constexpr (!kPair) {
-    // TMEM stores from warps 4..7 (lane quarter warp % 4), columns [384, 432)
-    if ((op == 8 || op == 9) && warp >= 4) {
-      uint32_t r32[32], r16[16];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) r32[j] = j;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) r16[j] = j;
-      const uint32_t lane_base = t + ((uint32_t)((warp & 3) * 32) << 16);
-      const unsigned long long t0 = clock64();
-      const int n = op == 8 ? iters : iters / 4;
-      for (int i = 0; i < n; ++i) {
-        tmem_st_32cols(lane_base + 384, r32);
-        if (op == 9) tmem_st_16cols(lane_base + 416, r16);
-        tmem_st_wait();
-      }
-      if ((threadIdx.x & 31) == 0) cycles[gridDim.x * (warp - 3) + blockIdx.x] = clock64() - t0;
-    }
   }
   if constexpr (kPair) {
     if (!issuer && threadIdx.x == 0) mbar_wait(&done_bar, 0, &abort_sh);
@@ -1352,7 +1309,7 @@ __device__ __forceinline__ void probe_body(int op, int iters, unsigned long long
   }
 }
 
-__global__ void __launch_bounds__(256, 1) tc_probe_kernel(int op, int iters, unsigned long long* cycles) {
+__global__ void __launch_bounds__(128, 1) tc_probe_kernel(int op, int iters, unsigned long long* cycles) {
   probe_body<false>(op, iters, cycles);
 }
 
@@ -1727,7 +1684,8 @@ svdq_status svdq_probe_cvt(const float* in, int64_t n, uint8_t* e2m1, uint8_t* e
 }
 
 svdq_status svdq_probe_tc(int op, int iters, int ctas, unsigned long long* cycles, svdq_stream stream) {
-  if (op < 0 || op > 10 || iters <= 0 || ctas <= 0 || !cycles) return SVDQ_ERR_INVALID_ARG;
+  if (op < 0 || op > 4 || iters <= 0 || iters > (1 << 24) || ctas <= 0 || ctas > 4096 || !cycles)
+    return SVDQ_ERR_INVALID_ARG;
   svdq_status st = device_ready();
   if (st != SVDQ_OK) return st;
   cudaError_t e = cudaFuncSetAttribute(dev::tc_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1736,8 +1694,8 @@ svdq_status svdq_probe_tc(int op, int iters, int ctas, unsigned long long* cycle
   e = cudaFuncSetAttribute(dev::tc_probe_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dev::kProbeSmem);
   if (e != cudaSuccess) return cuda_fail(e, "tc_probe_pair_kernel attribute");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (op == 1 || op == 10) dev::tc_probe_pair_kernel<<<(ctas + 1) / 2 * 2, 128, dev::kProbeSmem, s>>>(op, iters, cycles);
-  else dev::tc_probe_kernel<<<ctas, 256, dev::kProbeSmem, s>>>(op, iters, cycles);
+  if (op == 1) dev::tc_probe_pair_kernel<<<(ctas + 1) / 2 * 2, 128, dev::kProbeSmem, s>>>(op, iters, cycles);
+  else dev::tc_probe_kernel<<<ctas, 128, dev::kProbeSmem, s>>>(op, iters, cycles);
   return launch_status("tc_probe launch");
 }
 
@@ -1781,7 +1739,10 @@ svdq_status noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "svdq_linear_noalloc cudaGetDevice");
-  if (dev < 0 || dev >= 64) return SVDQ_ERR_UNSUPPORTED;
+  if (dev < 0 || dev >= 64) {
+    snprintf(g_last_error, sizeof(g_last_error), "svdq_linear_noalloc: device index %d outside 0..63", dev);
+    return SVDQ_ERR_UNSUPPORTED;
+  }
   std::lock_guard<std::mutex> lk(g_scratch_mu);
   if (!g_scratch_addr[dev]) {
     void* a = nullptr;

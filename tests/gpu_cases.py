@@ -115,12 +115,28 @@ def compare(pp: Prepared, X: np.ndarray, run: Run, rows=None, code_rows=None) ->
     err = sq.rel_fro(run.Y[rows], Yref)
     out["y_rel_err"] = err
     assert err <= Y_TOL, f"Y rel err {err}"
+    if len(rows) == M:
+        # every output tile on its own: a wrong tile cannot hide in the global norm
+        worst, where = tile_errors(run.Y, Yref)
+        out["y_worst_tile_rel_err"] = worst
+        out["y_worst_tile"] = where
+        assert worst <= Y_TOL, f"Y rel err {worst} in the {TILE_M}x{TILE_N} tile at {where}"
     return out
 
 
-def sample_rows(M: int, n: int = 96, seed: int = 0) -> np.ndarray:
-    rng = np.random.default_rng(seed)
-    edge = [0, 1, 31, 32, 127, 128, 129, M // 2, M - 129, M - 128, M - 2, M - 1]
-    rows = set(r for r in edge if 0 <= r < M)
-    rows.update(rng.choice(M, size=min(n, M), replace=False).tolist())
-    return np.array(sorted(rows))
+TILE_M, TILE_N = 128, 256
+
+
+def tile_errors(Y: np.ndarray, Yref: np.ndarray):
+    """Largest relative Frobenius error over the (TILE_M x TILE_N) output
+    tiles (ragged at the edges), and that tile's (row, column) origin."""
+    worst, where = 0.0, (0, 0)
+    for r0 in range(0, Y.shape[0], TILE_M):
+        for c0 in range(0, Y.shape[1], TILE_N):
+            a = Y[r0:r0 + TILE_M, c0:c0 + TILE_N]
+            b = Yref[r0:r0 + TILE_M, c0:c0 + TILE_N]
+            nb = np.linalg.norm(b)
+            e = float(np.linalg.norm(a - b) / nb) if nb > 0 else float(np.linalg.norm(a - b))
+            if e > worst:
+                worst, where = e, (r0, c0)
+    return worst, where

@@ -469,3 +469,25 @@ def pin_act_scale_in_prepare(sq):
     # fl32 of the exact quotient: within half an fp32 ulp of it
     ulp = Fraction(2) ** (math.frexp(float(expect))[1] - 24)
     assert abs(got - expect) <= ulp / 2, (float(got), float(expect))
+
+
+def pin_lapack_factors_match_jacobi(sq):
+    """The LAPACK route to the truncated factors gives the same rank-r
+    product as the oracle's Jacobi sweeps (both are the Eckart-Young optimum;
+    singular vectors may differ in sign, which cancels in L1 L2), so either
+    can prepare a layer: the products agree to the 16-bit rounding of the
+    factors, and the residual norms to the same order."""
+    rng = np.random.default_rng(19)
+    for (K, N, r, dt) in ((96, 80, 8, "bf16"), (64, 160, 16, "fp16")):
+        Wt = (rng.standard_normal((N, K)) / math.sqrt(K)).astype(np.float32)
+        x = rng.standard_normal((32, K)); x[:, [3, 40]] *= 50
+        _, lam = sq.smoothing_factors(x, Wt, 0.5)
+        W_hat = sq.smooth_weight(Wt, lam)
+        A1, A2, sa = sq.low_rank_factors(W_hat, r, dt, "jacobi")
+        B1, B2, sb = sq.low_rank_factors(W_hat, r, dt, "lapack")
+        assert np.max(np.abs(sa - sb)) <= 1e-12 * sa[0]
+        P, Q = A1 @ A2, B1 @ B2
+        u = 2.0 ** (-8 if dt == "bf16" else -11)
+        assert np.linalg.norm(P - Q) <= 4 * u * np.linalg.norm(P)
+        ra = np.linalg.norm(W_hat - P); rb = np.linalg.norm(W_hat - Q)
+        assert abs(ra - rb) <= 4 * u * np.linalg.norm(P)

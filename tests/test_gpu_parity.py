@@ -112,24 +112,24 @@ def test_repeat_calls_are_bitwise_identical(gpu, fmt):
 @pytest.mark.parametrize("name", ["flux_qkv_int4", "flux_ffn_up_nvfp4", "ffn_down_nvfp4", "ffn_down_int4"])
 def test_full_size_config(gpu, name):
     """Full-size FLUX / FFN-down layers in the benchmark's launch configuration:
-    codes on 512 sampled tokens and Y on ~100 sampled tokens (incl. tile edges)."""
+    every code and scale bit-exact, every output element of Y against the
+    oracle, globally and per 128 x 256 tile."""
     pp = G.prepared_preset(name)
     X = pp.wl.X
     run = G.run_gpu(pp, X)
-    M = X.shape[0]
-    res = G.compare(pp, X, run, rows=G.sample_rows(M), code_rows=G.sample_rows(M, 500, seed=1))
+    res = G.compare(pp, X, run)
     print(name, res)
 
 
 @pytest.mark.parametrize("shape", ["var_up_nvfp4", "var_down_nvfp4"])
 def test_var_token_sweep(gpu, shape):
-    """Infinity-VAR style projections at every token count of the sweep."""
+    """Infinity-VAR style projections at every token count of the sweep:
+    every code and every output element (globally and per tile)."""
     pp = G.prepared_preset(shape)
     for M in synth.VAR_TOKENS:
         X = pp.wl.X[:M]
         run = G.run_gpu(pp, X)
-        rows = G.sample_rows(M, 48)
-        G.compare(pp, X, run, rows=rows, code_rows=rows)
+        print(shape, M, G.compare(pp, X, run))
 
 
 def test_status_word_clean(gpu):

@@ -83,3 +83,7 @@ def test_act_codes_from_smoothed_x_golden():
 
 def test_act_tensor_scale_in_prepare():
     P.pin_act_scale_in_prepare(svdquant)
+
+
+def test_lapack_factors_match_jacobi():
+    P.pin_lapack_factors_match_jacobi(svdquant)

@@ -24,6 +24,10 @@
 //   ux   M x lrw bf16: [u'_hi | u'_lo (| u'_hi) | 0 pad], u' = u / (s_gX s_gW) (NVFP4) or u (INT4)
 //        (NVFP4: as low-rank tiles over Mp rows; INT4: row-major)
 //   part, cnt   NVFP4 K-split scratch when nvfp4_split_k_eligible (below), else empty
+//   upart, ucnt NVFP4 activation kernel K split (act_nv_ks > 1): fp32 partial down
+//               projections [Mp/128][ks][128][r] and one 64-bit arrival word per
+//               128-token tile (need no initial value: each call tags its
+//               arrivals with a fresh epoch)
 //
 // NVFP4 operand tiles (what one bulk copy brings into shared memory, ready
 // for the tensor core): 128 rows x one K slab of 256 elements.  The E2M1
@@ -106,7 +110,7 @@ inline BlobLayout blob_layout(const svdq_params& p) {
 }
 
 struct WsLayout {
-  size_t off_xq, off_xs, off_ux, off_part, off_cnt, total;
+  size_t off_xq, off_xs, off_ux, off_part, off_cnt, off_upart, off_ucnt, total;
   int64_t Mp;  // M rounded up to the GEMM's row tile (256 NVFP4, 128 INT4)
 };
 
@@ -117,6 +121,21 @@ struct WsLayout {
 constexpr int kMaxKSplit = 8;
 inline bool nvfp4_split_k_eligible(const svdq_params& p, int64_t M) {
   return p.fmt == SVDQ_NVFP4 && M >= 1 && M <= 64 && p.N / 256 <= 37;
+}
+
+// K split of the NVFP4 activation kernel: ks CTAs (a power of two dividing
+// K / 256, at most 16, which bounds the contention on a tile's arrival word)
+// share each 128-token tile so that the grid fills about the 148 SMs of a
+// B200.  A fixed function of the shape, so that the host sizes the workspace
+// the same way the launcher splits.
+constexpr int kActSizingSMs = 148;
+constexpr int kActMaxKs = 16;
+SVDQ_HD inline int act_nv_ks(int64_t Mp, int K) {
+  const int64_t tiles = Mp / 128;
+  const int slabs = K / 256;
+  int ks = 1;
+  while (ks < kActMaxKs && tiles * ks * 2 <= kActSizingSMs && slabs % (ks * 2) == 0) ks *= 2;
+  return ks;
 }
 
 inline WsLayout ws_layout(const svdq_params& p, int64_t M) {
@@ -138,6 +157,15 @@ inline WsLayout ws_layout(const svdq_params& p, int64_t M) {
     off = align_up(off + (size_t)kMaxKSplit * (size_t)M * (size_t)p.N * 4);
     L.off_cnt = off;
     off = align_up(off + (size_t)(p.N / 256) * (Mp / 256) * 16 * 4);
+  }
+  L.off_upart = L.off_ucnt = off;
+  if (p.fmt == SVDQ_NVFP4 && M > 256) {   // the 128-token-tile activation kernel (see the launcher)
+    const int ks = act_nv_ks(L.Mp, p.K);
+    if (ks > 1 && p.rank > 0) {
+      off = align_up(off + (Mp / 128) * (size_t)ks * 128 * (size_t)p.rank * 4);
+      L.off_ucnt = off;
+      off = align_up(off + (Mp / 128) * 8);
+    }
   }
   L.total = off > 0 ? off : kAlign;
   return L;

@@ -132,6 +132,13 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
                "r"(smem_u32(src)), "r"(x), "r"(y)
                : "memory");
 }
+// Plain bulk copy shared -> global (both 16-byte aligned, bytes % 16 == 0),
+// tracked by the issuing thread's bulk async-group.
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
+               "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void bulk_wait_read() {
@@ -182,6 +189,12 @@ __device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr_cluster) {
                : "r"(addr_cluster)
                : "memory");
   return v;
+}
+
+__device__ __forceinline__ void st_cluster_f32x4(uint32_t addr_cluster, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr_cluster), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
 }
 
 __device__ __forceinline__ void st_cluster_u32(uint32_t addr_cluster, uint32_t v) {
@@ -411,6 +424,13 @@ __host__ __device__ constexpr uint32_t idesc_f16_bf16(int M, int N) {
   return (1u << 4)                 // D format: f32
          | (1u << 7)               // A: bf16
          | (1u << 10)              // B: bf16
+         | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__host__ __device__ constexpr uint32_t idesc_f16_f16(int M, int N) {
+  return (1u << 4)                 // D format: f32
+         | (0u << 7)               // A: f16
+         | (0u << 10)              // B: f16
          | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 

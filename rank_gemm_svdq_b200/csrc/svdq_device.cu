@@ -25,6 +25,8 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <mutex>
 #include <vector>
 
@@ -564,6 +566,435 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
       record_status(kStatusTimeout);
       return;
     }
+  }
+}
+
+// ------------------------------------------------------------ kernel 1, NVFP4 form
+// NVFP4 activations on 128-token tiles (one TMEM lane per token), with the K
+// range of a tile split over ks CTAs (act_nv_ks) so that the grid fills the
+// SMs.  Per 128-wide half of a 256-wide K slab (one ring stage):
+//   producer   TMA-loads the X half slab (128 tokens x 128: two 128-byte-
+//              swizzled atoms), the matching L1^T columns and inv_lambda;
+//   quantiser  16 warps; warp w owns 16-element block w % 8 of the half for
+//              tokens 64 (w / 8) + lane + {0, 32}: X^ = fp32(x) * inv_lambda,
+//              block amax -> E4M3 scale -> E2M1 codes, written straight into
+//              the GEMM's activation tile in shared memory; X^ rounded to the
+//              16-bit dtype overwrites x in place, which makes the stage the A
+//              operand of the down projection;
+//   MMA thread issues u += X^16 L1 on tcgen05 (M = 128 tokens, N = r, fp32 in
+//              TMEM), frees the stage, and once both halves of a slab are
+//              quantised writes the 18 KB activation tile out with one bulk copy.
+// After the last slab four warps read the partial u from TMEM.  With ks = 1
+// they write u' = u / (s_gX s_gW) as bf16 hi + lo into the low-rank input
+// tile.  With ks > 1 every CTA writes its partial to the workspace and
+// counts in on its tile's arrival word (tagged with this call's epoch, so no
+// initial value is needed); the last CTA to arrive adds the ks partials in K
+// order (deterministic), writes u' and clears the word.  Tokens past M stay
+// zero (TMA fills them, and zeros quantise to zero codes and scale 0).
+struct ActNvArgs {
+  int64_t M, Mp;
+  int K, r, lrw, nseg;
+  int slabs;          // 256-wide K slabs per CTA
+  int ks;             // CTAs per 128-token tile (K split)
+  int stages;         // ring depth
+  unsigned long long epoch;   // nonzero, distinct per call (K split arrivals)
+  const float* inv_lambda;
+  const BlobHeader* hdr;
+  uint8_t* xq;        // activation tiles [Mp/128][K/256]
+  uint8_t* ux;        // low-rank input tiles [Mp/128][lrw/64]
+  float* upart;       // ks > 1: partial u [Mp/128][ks][128][r]
+  unsigned long long* ucnt;   // ks > 1: arrival word per 128-token tile
+  int* gemm_cnt;      // GEMM K-split arrival counters to clear (or null)
+  int n_cnt;
+};
+
+constexpr int kAN_Quant = 16;
+constexpr int kAN_Threads = (2 + kAN_Quant) * 32;
+constexpr int kAN_XBytes = 128 * 128 * 2;        // X half slab: two 16 KB atoms
+constexpr int kAN_IlBytes = 128 * 4;             // inv_lambda of the half slab
+constexpr int kAN_Budget = 232448 - 4096;        // dynamic shared memory budget (static tables aside)
+constexpr int kAN_MaxStages = 6;
+
+// stage: [X atoms | L1^T atoms (2 x r rows x 128 bytes) | inv_lambda], 1024-aligned
+SVDQ_HD inline int an_stage_bytes(int r) { return (kAN_XBytes + 2 * r * 128 + kAN_IlBytes + 1023) / 1024 * 1024; }
+SVDQ_HD inline int an_stages(int r) {
+  const int s = (kAN_Budget - 1024 - 2 * kATile) / an_stage_bytes(r);
+  return s > kAN_MaxStages ? kAN_MaxStages : s;
+}
+SVDQ_HD inline int an_smem_bytes(int r) { return 1024 + an_stages(r) * an_stage_bytes(r) + 2 * kATile; }
+
+// One NVFP4 block of 16 smoothed activations -> 8 code bytes (p0, p1) and
+// the E4M3 scale code (same arithmetic as quantize16).
+__device__ __forceinline__ void nv_block(const float (&xh)[16], float six_sg, float r6, const float* dq,
+                                         uint32_t& p0, uint32_t& p1, uint32_t& e) {
+  float m8[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fabsf(xh[i]), fabsf(xh[i + 8]));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m8[i] = fmaxf(m8[i], m8[i + 4]);
+  const float amax = fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3]));
+  const float ratio = r6 != 0.0f ? div_by_recip(amax, six_sg, r6) : __fdiv_rn(amax, six_sg);
+  e = cvt_e4m3x2(0.0f, ratio) & 0xFFu;
+  const float d = dq[e];
+  const float rd = dq[256 + e];
+  p0 = 0; p1 = 0;
+  if (d != 0.0f) {
+    if (rd != 0.0f) {
+      const uint64_t nd2 = f2_pack(-d, -d), r2 = f2_pack(rd, rd);
+      uint32_t b[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float q0, q1;
+        f2_unpack(div2_by_recip(f2_pack(xh[2 * i], xh[2 * i + 1]), nd2, r2), q0, q1);
+        b[i] = cvt_e2m1x2(q1, q0);
+      }
+      p0 = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+      p1 = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        p0 |= cvt_e2m1x2(__fdiv_rn(xh[2 * i + 1], d), __fdiv_rn(xh[2 * i], d)) << (8 * i);
+        p1 |= cvt_e2m1x2(__fdiv_rn(xh[2 * i + 9], d), __fdiv_rn(xh[2 * i + 8], d)) << (8 * i);
+      }
+    }
+  }
+}
+
+template <int DT>
+__device__ __forceinline__ void unpack8(const uint4 v, float* f) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if constexpr (DT == SVDQ_BF16) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    } else {
+      const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+      f[2 * i] = t.x;
+      f[2 * i + 1] = t.y;
+    }
+  }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kAN_Threads, 1)
+    act_nvfp4_kernel(const ActNvArgs a, const __grid_constant__ CUtensorMap tm_x,
+                     const __grid_constant__ CUtensorMap tm_l1) {
+  extern __shared__ __align__(1024) uint8_t an_raw[];
+  __shared__ uint64_t full_bar[kAN_MaxStages], empty_bar[kAN_MaxStages], qdone_bar[kAN_MaxStages];
+  __shared__ uint64_t tfree_bar[2], accf_bar;
+  __shared__ uint32_t tmem_sh;
+  __shared__ int abort_sh, last_sh;
+  __shared__ float dq_tab[512];
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(an_raw) + 1023) & ~uintptr_t(1023));
+  const int S = a.stages, r = a.r;
+  const int sbytes = an_stage_bytes(r);
+  const int off_il = kAN_XBytes + 2 * r * 128;
+  const uint32_t stage_tx = (uint32_t)(kAN_XBytes + 2 * r * 128 + kAN_IlBytes);
+  uint8_t* ctile = smem + S * sbytes;            // two activation tiles being assembled
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int KS = a.ks;
+  const int kq = blockIdx.x % KS;                // K part of the tile
+  const int mtile = blockIdx.x / KS;             // 128-token tile
+  const int64_t m0 = (int64_t)mtile * 128;
+  const int slab0 = kq * a.slabs;
+  const int nhalf = 2 * a.slabs;
+  const int ksl = a.K / 256;
+  const uint32_t tcols = r <= 32 ? 32u : (r <= 64 ? 64u : 128u);
+  // a tile wholly past the last token (M rounded up to the GEMM's 256 rows)
+  // loads nothing: its activation tiles and low-rank rows are written as zeros
+  const bool live_tile = m0 < a.M;
+  const int rows_live = live_tile ? (int)(a.M - m0 < 128 ? a.M - m0 : 128) : 0;
+  volatile int* abort_flag = &abort_sh;
+
+  griddep_launch();   // the GEMM may start its prologue on idle SMs
+  // ring stage c: X half slab, L1^T columns and inv_lambda at K offset (2 slab0 + c) * 128
+  auto issue_half = [&](int c) {
+    const int s = c % S;
+    uint8_t* st = smem + s * sbytes;
+    const int k0 = slab0 * 256 + c * 128;
+    mbar_arrive_expect_tx(&full_bar[s], stage_tx);
+    tma_load_2d(st, &tm_x, &full_bar[s], k0, (int)m0);
+    tma_load_2d(st + 16384, &tm_x, &full_bar[s], k0 + 64, (int)m0);
+    if (r > 0) {
+      tma_load_2d(st + kAN_XBytes, &tm_l1, &full_bar[s], k0, 0);
+      tma_load_2d(st + kAN_XBytes + r * 128, &tm_l1, &full_bar[s], k0 + 64, 0);
+    }
+    bulk_load(st + off_il, a.inv_lambda + k0, kAN_IlBytes, &full_bar[s]);
+  };
+  const int first = nhalf < S ? nhalf : S;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); mbar_init(&qdone_bar[s], kAN_Quant);
+    }
+    mbar_init(&tfree_bar[0], 1); mbar_init(&tfree_bar[1], 1);
+    mbar_init(&accf_bar, 1);
+    abort_sh = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+    if (live_tile)   // the first stages load while the rest of the CTA sets up
+      for (int c = 0; c < first; ++c) issue_half(c);
+  }
+  const float s_gx = a.hdr->s_gx;
+  if (threadIdx.x < 256) {
+    const float d = __fmul_rn(e4m3_val((uint32_t)threadIdx.x), s_gx);
+    dq_tab[threadIdx.x] = d;
+    dq_tab[256 + threadIdx.x] = (d != 0.0f && recip_ok(d)) ? __frcp_rn(d) : 0.0f;
+  }
+  if (rows_live < 128)   // rows past M keep zero codes and scales (never written below)
+    for (int i = threadIdx.x; i < 2 * kATile / 16; i += kAN_Threads)
+      reinterpret_cast<uint4*>(ctile)[i] = make_uint4(0, 0, 0, 0);
+  if (blockIdx.x == 0 && a.gemm_cnt)
+    for (int i = threadIdx.x; i < a.n_cnt; i += kAN_Threads) a.gemm_cnt[i] = 0;
+  if (warp == 1) { tmem_alloc(&tmem_sh, tcols); tmem_relinquish(); }
+  fence_proxy_async_smem();   // zeroed tiles are read by bulk copies
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_sh;
+  uint8_t* const xq_tile = a.xq + (size_t)mtile * ksl * kATile;   // + slab * kATile
+
+  if (!live_tile) {
+    if (warp == 1 && lane == 0) {
+      for (int t = 0; t < a.slabs; ++t) bulk_store(xq_tile + (size_t)(slab0 + t) * kATile, ctile, kATile);
+      bulk_commit();
+      bulk_wait_all();
+    }
+  } else if (warp == 0) {
+    if (lane == 0) {
+      int issued = first;
+      for (int c = first; c < nhalf; ++c) {
+        const int s = c % S;
+        if (!mbar_wait(&empty_bar[s], ((c / S) & 1) ^ 1, abort_flag)) break;
+        issue_half(c);
+        issued = c + 1;
+      }
+      if (*abort_flag)
+        for (int i = issued - 1; i >= 0 && i >= issued - S; --i) mbar_drain(&full_bar[i % S], (i / S) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = DT == SVDQ_BF16 ? idesc_f16_bf16(128, r) : idesc_f16_f16(128, r);
+      bool dead = false;
+      for (int c = 0; c < nhalf; ++c) {
+        const int s = c % S;
+        if (!mbar_wait(&qdone_bar[s], (c / S) & 1, abort_flag)) { dead = true; break; }
+        tc_fence_after();
+        if (r > 0) {
+          const uint32_t a_addr = smem_u32(smem + s * sbytes);
+          const uint32_t b_addr = a_addr + kAN_XBytes;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              mma_f16(tbase, desc_k_sw128(a_addr + h * 16384 + 32 * q), desc_k_sw128(b_addr + h * r * 128 + 32 * q),
+                      idesc, (c | h | q) != 0);
+        }
+        mma_commit(&empty_bar[s]);
+        if (c & 1) {
+          // both halves of slab t are in the tile buffer: one bulk copy out
+          const int t = c >> 1;
+          bulk_store(xq_tile + (size_t)(slab0 + t) * kATile, ctile + (t & 1) * kATile, kATile);
+          bulk_commit();
+          bulk_wait_read<0>();
+          mbar_arrive(&tfree_bar[t & 1]);
+        }
+      }
+      mma_commit(&accf_bar);
+      if (dead) mbar_drain(&accf_bar, 0);
+      bulk_wait_all();
+    }
+  } else {
+    // quantiser warps
+    const int qw = warp - 2;
+    const int jb = qw & 7;                         // 16-element block inside the half slab
+    const int row0 = (qw >> 3) * 64 + lane;        // tokens row0 and row0 + 32 of the tile
+    const int cc = (jb & 3) * 2;                   // its first 16-byte chunk in a 128-byte atom row
+    const float six_sg = __fmul_rn(6.0f, s_gx);
+    const float r6 = recip_ok(six_sg) ? __frcp_rn(six_sg) : 0.0f;
+    // rows of this warp past the last token are zero and stay unquantised
+    const int nrow = (qw >> 3) * 64 < rows_live ? ((qw >> 3) * 64 + 32 < rows_live ? 2 : 1) : 0;
+    for (int c = 0; c < nhalf; ++c) {
+      const int s = c % S, t = c >> 1, h = c & 1;
+      if (h == 0 && t >= 2)
+        if (!mbar_wait(&tfree_bar[t & 1], ((t >> 1) - 1) & 1, abort_flag)) break;
+      if (!mbar_wait(&full_bar[s], (c / S) & 1, abort_flag)) break;
+      uint8_t* st = smem + s * sbytes;
+      float il[16];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 f = reinterpret_cast<const float4*>(st + off_il)[4 * jb + i];
+        il[4 * i] = f.x; il[4 * i + 1] = f.y; il[4 * i + 2] = f.z; il[4 * i + 3] = f.w;
+      }
+      uint8_t* xatom = st + (jb >> 2) * 16384;
+      uint8_t* tileb = ctile + (t & 1) * kATile;
+      const int j16 = 8 * h + jb;                  // block inside the 256-wide slab
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        if (i >= nrow) break;
+        const int row = row0 + 32 * i;
+        uint8_t* rowp = xatom + row * 128;
+        uint4* c0p = reinterpret_cast<uint4*>(rowp + ((cc ^ (row & 7)) << 4));
+        uint4* c1p = reinterpret_cast<uint4*>(rowp + (((cc + 1) ^ (row & 7)) << 4));
+        float xf[16];
+        unpack8<DT>(*c0p, xf);
+        unpack8<DT>(*c1p, xf + 8);
+        float xh[16];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          f2_unpack(f2_mul(f2_pack(xf[2 * k], xf[2 * k + 1]), f2_pack(il[2 * k], il[2 * k + 1])), xh[2 * k],
+                    xh[2 * k + 1]);
+        uint32_t p0, p1, e;
+        nv_block(xh, six_sg, r6, dq_tab, p0, p1, e);
+        *reinterpret_cast<uint2*>(tileb + sw128((uint32_t)row, 8u * (uint32_t)j16)) = make_uint2(p0, p1);
+        tileb[kTileCodes + tile_sf((uint32_t)row, (uint32_t)j16)] = (uint8_t)e;
+        uint4 o0, o1;
+        o0.x = pack_half2_rn<DT>(xh[0], xh[1]);   o0.y = pack_half2_rn<DT>(xh[2], xh[3]);
+        o0.z = pack_half2_rn<DT>(xh[4], xh[5]);   o0.w = pack_half2_rn<DT>(xh[6], xh[7]);
+        o1.x = pack_half2_rn<DT>(xh[8], xh[9]);   o1.y = pack_half2_rn<DT>(xh[10], xh[11]);
+        o1.z = pack_half2_rn<DT>(xh[12], xh[13]); o1.w = pack_half2_rn<DT>(xh[14], xh[15]);
+        *c0p = o0;
+        *c1p = o1;
+      }
+      fence_proxy_async_smem();   // X^16 and the tile are read by the tensor core and a bulk copy
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qdone_bar[s]);
+    }
+  }
+
+  // ---- partial u: TMEM -> the workspace (ks > 1) or shared memory (ks = 1),
+  // live rows only (warps 2..5, one TMEM lane quarter each)
+  const bool epi = warp >= 2 && warp < 6;
+  const int rs = r + 4;                            // row stride of the shared-memory copy
+  if (epi && r > 0 && live_tile && __all_sync(0xffffffffu, mbar_wait(&accf_bar, 0, abort_flag))) {
+    tc_fence_after();
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    float* part = a.upart + (((size_t)mtile * KS + kq) * 128 + row) * r;
+    for (int c0 = 0; c0 < r; c0 += 16) {
+      uint32_t v[16];
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+          "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+            "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+          : "r"(tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)c0));
+      tmem_ld_wait();
+      if (row < rows_live) {
+        float4* dst = KS > 1 ? reinterpret_cast<float4*>(part + c0)
+                             : reinterpret_cast<float4*>(reinterpret_cast<float*>(smem) + row * rs + c0);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float4 f = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                       __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
+          if (KS > 1) __stcg(dst + k, f); else dst[k] = f;
+        }
+      }
+    }
+    if (KS > 1) __threadfence();   // the partial is visible before this CTA counts in
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, tcols);
+  }
+  // ---- K split: count in; the last CTA of the tile adds the partials
+  bool finisher = true;
+  if (KS > 1 && r > 0 && live_tile) {
+    if (threadIdx.x == 64) {
+      __threadfence();
+      unsigned long long* w = a.ucnt + mtile;
+      unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(w), seen;
+      int last = 0;
+      for (;;) {
+        const bool same = (old >> 8) == a.epoch;
+        const unsigned long long cnt = same ? (old & 0xFF) : 0ull;
+        const unsigned long long next = (cnt + 1 == (unsigned long long)KS) ? 0ull : ((a.epoch << 8) | (cnt + 1));
+        seen = atomicCAS(w, old, next);
+        if (seen == old) { last = cnt + 1 == (unsigned long long)KS; break; }
+        old = seen;
+      }
+      last_sh = last;
+    }
+    __syncthreads();
+    finisher = last_sh != 0;
+    if (finisher) __threadfence();
+  }
+  if (!finisher || a.lrw == 0) return;
+  // ---- u' = u / (s_gX s_gW) as bf16 hi + lo into the low-rank input tile.
+  // Work items are (live row, 4 columns); a group of `lpi` lanes shares an
+  // item, lane i of the group adding partials i, i + lpi, ... in K order, and
+  // the group combines its lanes with a fixed shuffle tree (the same order on
+  // every call for a given shape).
+  const float inv_alpha = 1.0f / (a.hdr->s_gx * a.hdr->s_gw);
+  uint8_t* utiles = a.ux + (size_t)mtile * (a.lrw / 64) * kLRTile;
+  auto store4 = [&](int row, int col, uint32_t w0, uint32_t w1) {   // 4 bf16 at columns col..col+3
+    uint8_t* tile = utiles + (size_t)(col / 64) * kLRTile;
+    *reinterpret_cast<uint2*>(tile + sw128((uint32_t)row, (uint32_t)(col % 64) * 2)) = make_uint2(w0, w1);
+  };
+  const int c4 = r / 4;
+  const int items = rows_live * c4;
+  int lpi = 1;
+  if (KS > 1)
+    while (lpi < 32 && lpi < KS && items * lpi * 2 <= kAN_Threads) lpi *= 2;
+  const int groups = kAN_Threads / lpi;
+  const int gid = (int)threadIdx.x / lpi, gl = (int)threadIdx.x % lpi;
+  for (int it0 = 0; it0 < items; it0 += groups) {   // uniform trip count: the shuffles need every lane
+    const int it = it0 + gid;
+    const bool act = it < items;
+    const int row = act ? it / c4 : 0, col = act ? (it % c4) * 4 : 0;
+    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (act) {
+      if (KS > 1) {
+        // this lane's partials (at most kActMaxKs / lpi), all loads in flight before the K-ordered sum
+        const float* base = a.upart + ((size_t)mtile * KS * 128 + row) * r + col;
+        const int nsrc = (KS - gl + lpi - 1) / lpi;
+        for (int b0 = 0; b0 < nsrc; b0 += 4) {
+          float4 w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (b0 + i < nsrc) w[i] = __ldcg(reinterpret_cast<const float4*>(base + (size_t)(gl + (b0 + i) * lpi) * 128 * r));
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (b0 + i < nsrc) { u.x += w[i].x; u.y += w[i].y; u.z += w[i].z; u.w += w[i].w; }
+        }
+      } else {
+        u = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(smem) + row * rs + col);
+      }
+    }
+    for (int off = 1; off < lpi; off <<= 1) {
+      u.x += __shfl_xor_sync(0xffffffffu, u.x, off);
+      u.y += __shfl_xor_sync(0xffffffffu, u.y, off);
+      u.z += __shfl_xor_sync(0xffffffffu, u.z, off);
+      u.w += __shfl_xor_sync(0xffffffffu, u.w, off);
+    }
+    if (act && gl == 0) {
+      const float v[4] = {u.x * inv_alpha, u.y * inv_alpha, u.z * inv_alpha, u.w * inv_alpha};
+      uint32_t hi[2], lo[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const uint32_t h0 = bf16_rn(v[2 * k]), h1 = bf16_rn(v[2 * k + 1]);
+        const uint32_t l0 = bf16_rn(v[2 * k] - __uint_as_float(h0 << 16));
+        const uint32_t l1 = bf16_rn(v[2 * k + 1] - __uint_as_float(h1 << 16));
+        hi[k] = h0 | (h1 << 16);
+        lo[k] = l0 | (l1 << 16);
+      }
+      store4(row, col, hi[0], hi[1]);
+      store4(row, r + col, lo[0], lo[1]);
+      if (a.nseg == 3) store4(row, 2 * r + col, hi[0], hi[1]);
+    }
+  }
+  // zero padding columns of the live rows and every column of the rows past M
+  const int pad0 = a.nseg * r;
+  const int npad = (a.lrw - pad0) / 4;
+  const int zitems = rows_live * npad + (128 - rows_live) * (a.lrw / 4);
+  for (int it = threadIdx.x; it < zitems; it += kAN_Threads) {
+    int row, col;
+    if (it < rows_live * npad) { row = it / npad; col = pad0 + (it % npad) * 4; }
+    else { const int j = it - rows_live * npad; row = rows_live + j / (a.lrw / 4); col = (j % (a.lrw / 4)) * 4; }
+    store4(row, col, 0u, 0u);
   }
 }
 
@@ -1426,7 +1857,11 @@ svdq_status device_ready() {
              cudaFuncSetAttribute(dev::act_quant_kernel<SVDQ_INT4_G64, SVDQ_BF16>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, act_smem) == cudaSuccess &&
              cudaFuncSetAttribute(dev::act_quant_kernel<SVDQ_INT4_G64, SVDQ_F16>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, act_smem) == cudaSuccess;
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, act_smem) == cudaSuccess &&
+             cudaFuncSetAttribute(dev::act_nvfp4_kernel<SVDQ_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  dev::kAN_Budget) == cudaSuccess &&
+             cudaFuncSetAttribute(dev::act_nvfp4_kernel<SVDQ_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  dev::kAN_Budget) == cudaSuccess;
       d.ok = d.ok && encoder();
     }
   }
@@ -1461,6 +1896,11 @@ int act_k_split(int64_t Mp, int K) {
   while (ks < 8 && groups * ks * 2 <= num_sms() && chunks % (ks * 2) == 0) ks *= 2;
   return ks;
 }
+
+// Per-call tag of the activation kernel's K-split arrivals (56 bits, never 0),
+// started from the clock so that another process's leftovers never match.
+std::atomic<unsigned long long> g_act_epoch{
+    ((unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count() * 0x9E3779B97F4A7C15ull) >> 8};
 
 template <int FMT>
 cudaError_t launch_act(const svdq_params* p, dev::ActArgs a, int64_t Mp, cudaStream_t stream) {
@@ -1513,6 +1953,46 @@ svdq_status launch_quantize(const svdq_params* p, const void* blob_dev, const vo
   a.ux = reinterpret_cast<uint16_t*>(ws + W.off_ux);
   a.gemm_cnt = W.off_cnt > W.off_part ? reinterpret_cast<int*>(ws + W.off_cnt) : nullptr;
   a.n_cnt = (p->N / 256) * (int)(W.Mp / 256) * 16;
+  // NVFP4 above 256 tokens: the 128-token-tile kernel (tcgen05 down projection).
+  // Up to 256 tokens the 32-token kernel wins: its latency chain per call is
+  // shorter (measured 12-22 us against 20-25 us at one token on the VAR shapes).
+  if (p->fmt == SVDQ_NVFP4 && M > 256) {
+    dev::ActNvArgs n;
+    n.M = M; n.Mp = W.Mp; n.K = p->K; n.r = p->rank; n.lrw = lr_width(*p); n.nseg = nseg_of(*p);
+    n.ks = act_nv_ks(W.Mp, p->K);
+    n.slabs = p->K / 256 / n.ks;
+    n.stages = dev::an_stages(p->rank);
+    n.epoch = g_act_epoch.fetch_add(1) & 0x00FFFFFFFFFFFFFFull;
+    if (n.epoch == 0) n.epoch = g_act_epoch.fetch_add(1) & 0x00FFFFFFFFFFFFFFull;
+    n.inv_lambda = a.inv_lambda;
+    n.hdr = a.hdr;
+    n.xq = a.xq;
+    n.ux = reinterpret_cast<uint8_t*>(a.ux);
+    n.upart = reinterpret_cast<float*>(ws + W.off_upart);
+    n.ucnt = reinterpret_cast<unsigned long long*>(ws + W.off_ucnt);
+    n.gemm_cnt = a.gemm_cnt;
+    n.n_cnt = a.n_cnt;
+    const CUtensorMapDataType dt =
+        p->act_dtype == SVDQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUtensorMap tm_x, tm_l1;
+    bool ok = make_map(&tm_x, dt, X, (uint64_t)p->K, (uint64_t)M, (uint64_t)p->K * 2, 64, 128);
+    if (p->rank > 0)
+      ok = ok && make_map(&tm_l1, dt, a.l1t, (uint64_t)p->K, (uint64_t)p->rank, (uint64_t)p->K * 2, 64,
+                          (uint32_t)p->rank);
+    else
+      tm_l1 = tm_x;   // not read at rank 0
+    if (!ok) return cuda_fail(cudaErrorInvalidValue, "tensor map encode (activation kernel)");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(W.Mp / 128 * n.ks));
+    cfg.blockDim = dim3(dev::kAN_Threads);
+    cfg.dynamicSmemBytes = (size_t)dev::an_smem_bytes(p->rank);
+    cfg.stream = stream;
+    const cudaError_t e = p->act_dtype == SVDQ_BF16
+                              ? cudaLaunchKernelEx(&cfg, dev::act_nvfp4_kernel<SVDQ_BF16>, n, tm_x, tm_l1)
+                              : cudaLaunchKernelEx(&cfg, dev::act_nvfp4_kernel<SVDQ_F16>, n, tm_x, tm_l1);
+    if (e != cudaSuccess) return cuda_fail(e, "act_nvfp4_kernel launch");
+    return launch_status("act_nvfp4_kernel launch");
+  }
   const cudaError_t e = p->fmt == SVDQ_NVFP4 ? launch_act<SVDQ_NVFP4>(p, a, W.Mp, stream)
                                              : launch_act<SVDQ_INT4_G64>(p, a, W.Mp, stream);
   if (e != cudaSuccess) return cuda_fail(e, "act_quant_kernel launch");

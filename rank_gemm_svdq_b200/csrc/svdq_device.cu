@@ -1354,6 +1354,222 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
   }
 }
 
+// ------------------------------------------------------------ kernel 2, NVFP4, few tokens
+// Up to 16 tokens: the layer streams its weights, so the weight tile is the
+// 128-row A operand of a 1-CTA kind::mxf4nvf4 MMA and the tokens are a
+// 16-column B operand (M = 128 output features, N = 16 tokens, K = 64):
+// D[feature, token] accumulates in 16 TMEM columns.  One CTA per (128-feature
+// tile, K part); with ks > 1 K parts add through fp32 partials (the last CTA
+// of a tile adds them in K order, as in the pair kernel).
+// Per 256-wide K slab a ring stage holds the tile's codes (16 KB) and its
+// 128 rows of scale atoms (2 KB), and the first 16 rows of the activation
+// tile's codes (2 KB) and its scale atoms (2 KB): four bulk copies.  The
+// weight halves of the first stages are issued before the wait for the
+// activation kernel.  Four scale warps (one per TMEM lane quarter) move a
+// landed stage's eight scale atoms to its TMEM slot with tcgen05.st and
+// release it to the MMA thread, which then only issues the stage's four MMAs
+// (with the scale copies on the MMA thread, the measured issue cost was
+// ~0.5 us per stage, slower than the weight stream).  The low-rank up
+// projection u' L2 runs last as kind::f16 K-steps (A = the L2 tile of the 128
+// features, B = the first 16 rows of the low-rank input tile) into the same
+// accumulator.
+// Warps: 0 producer, 1 TMEM owner + MMA issuer, 2-5 scale warps, then the
+// epilogue (lane quarters).
+constexpr int kSM_Tokens = 16;
+constexpr int kSM_Stage = kTileCodes + 2048 + kSM_Tokens * 128 + 2048;   // 22528
+constexpr int kSM_Stages = 9;
+constexpr int kSM_Threads = 6 * 32;
+constexpr int kSM_Smem = kSM_Stages * kSM_Stage + 1024;
+// stage offsets: [W codes | W scales | X codes (16 rows) | X scales]
+constexpr int kSM_WS = kTileCodes, kSM_X = kTileCodes + 2048, kSM_XS = kSM_X + kSM_Tokens * 128;
+
+__global__ void __launch_bounds__(kSM_Threads, 1)
+    gemm_nvfp4_small_kernel(const PairArgs g) {
+  extern __shared__ __align__(1024) uint8_t gsmem_raw[];
+  __shared__ uint64_t full_bar[kSM_Stages], empty_bar[kSM_Stages], ready_bar[kSM_Stages], accf_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ks = g.ks;
+  const int nt = blockIdx.x / ks, kq = blockIdx.x % ks;
+  const int ksl = g.K / 256;
+  const int cpk = g.k_iters / ks;                 // slabs of this CTA: [kq cpk, (kq + 1) cpk)
+  const int lr = kq == 0 ? g.lr_iters : 0;        // the low-rank steps ride with K part 0
+  const int steps = cpk + lr;
+  volatile int* abort_flag = &abort_sh;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSM_Stages; ++s) {
+      mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); mbar_init(&ready_bar[s], 4);
+    }
+    mbar_init(&accf_bar, 1);
+    abort_sh = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) { tmem_alloc(&tmem_base_sh, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_base_sh;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // step j < cpk: slab kq cpk + j; step j >= cpk: low-rank K step j - cpk
+      auto weight_part = [&](int j, uint8_t* st) {
+        if (j < cpk) {
+          const uint8_t* wt = g.wtiles + ((size_t)nt * ksl + (size_t)(kq * cpk + j)) * kWTile;
+          bulk_load(st, wt, kTileCodes, &full_bar[j % kSM_Stages]);
+          bulk_load(st + kSM_WS, wt + kTileCodes + 2048 * (nt & 1), 2048, &full_bar[j % kSM_Stages]);
+        } else {
+          bulk_load(st, g.l2tiles + ((size_t)nt * g.lr_iters + (j - cpk)) * kLRTile, kLRTile,
+                    &full_bar[j % kSM_Stages]);
+        }
+      };
+      auto act_part = [&](int j, uint8_t* st) {
+        if (j < cpk) {
+          const uint8_t* at = g.atiles + (size_t)(kq * cpk + j) * kATile;   // tokens 0..127, slab
+          bulk_load(st + kSM_X, at, kSM_Tokens * 128, &full_bar[j % kSM_Stages]);
+          bulk_load(st + kSM_XS, at + kTileCodes, 2048, &full_bar[j % kSM_Stages]);
+        } else {
+          bulk_load(st + kSM_X, g.utiles + (size_t)(j - cpk) * kLRTile, kSM_Tokens * 128, &full_bar[j % kSM_Stages]);
+        }
+      };
+      auto stage_bytes = [&](int j) -> uint32_t {
+        return j < cpk ? (uint32_t)(kTileCodes + 2048 + kSM_Tokens * 128 + 2048) : (uint32_t)(kLRTile + kSM_Tokens * 128);
+      };
+      // the weights do not depend on the activation kernel: start them now
+      const int first = steps < kSM_Stages ? steps : kSM_Stages;
+      for (int j = 0; j < first; ++j) {
+        mbar_arrive_expect_tx(&full_bar[j], stage_bytes(j));
+        weight_part(j, smem + j * kSM_Stage);
+      }
+      griddep_wait();   // activation tiles and low-rank rows come from the activation kernel
+      for (int j = 0; j < first; ++j) act_part(j, smem + j * kSM_Stage);
+      int issued = first;
+      for (int j = first; j < steps; ++j) {
+        const int s = j % kSM_Stages;
+        if (!mbar_wait(&empty_bar[s], ((j / kSM_Stages) & 1) ^ 1, abort_flag)) break;
+        uint8_t* st = smem + s * kSM_Stage;
+        mbar_arrive_expect_tx(&full_bar[s], stage_bytes(j));
+        weight_part(j, st);
+        act_part(j, st);
+        issued = j + 1;
+      }
+      if (*abort_flag)
+        for (int i = issued - 1; i >= 0 && i >= issued - kSM_Stages; --i)
+          mbar_drain(&full_bar[i % kSM_Stages], (i / kSM_Stages) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_f4 = idesc_nvf4(128, kSM_Tokens);
+      const uint32_t id_lr = idesc_f16_bf16(128, kSM_Tokens);
+      bool dead = false;
+      for (int j = 0; j < steps; ++j) {
+        const int s = j % kSM_Stages;
+        // ready: the scale warps saw the stage land and wrote its scale slot
+        if (!mbar_wait(&ready_bar[s], (j / kSM_Stages) & 1, abort_flag)) { dead = true; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + s * kSM_Stage);
+        const uint32_t b_addr = a_addr + kSM_X;
+        if (j < cpk) {
+          const uint32_t sfa_t = tbase + 32 + 32 * s, sfb_t = sfa_t + 16;   // the stage's scale slot
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            mma_nvf4(tbase, desc_k_sw128(a_addr + 32 * q), desc_k_sw128(b_addr + 32 * q), id_f4, sfa_t + 4 * q,
+                     sfb_t + 4 * q, (j | q) != 0);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            mma_f16(tbase, desc_k_sw128(a_addr + 32 * q), desc_k_sw128(b_addr + 32 * q), id_lr, (j | q) != 0);
+        }
+        mma_commit(&empty_bar[s]);
+      }
+      mma_commit(&accf_bar);
+      if (dead) mbar_drain(&accf_bar, 0);
+    }
+  } else {
+    const int q = warp & 3;
+    // scale warps: a landed stage's scale atoms -> this lane quarter of its TMEM slot
+    {
+      const uint32_t lane_base = tbase + ((uint32_t)(q * 32) << 16);
+      for (int j = 0; j < steps; ++j) {
+        const int s = j % kSM_Stages;
+        if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[s], (j / kSM_Stages) & 1, abort_flag))) break;
+        if (j < cpk) {
+          const uint8_t* st = smem + s * kSM_Stage;
+          uint32_t w[16];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint4 a4 = *reinterpret_cast<const uint4*>(st + kSM_WS + 512 * k + lane * 16);
+            w[4 * k] = a4.x; w[4 * k + 1] = a4.y; w[4 * k + 2] = a4.z; w[4 * k + 3] = a4.w;
+          }
+          tc_fence_after();
+          tmem_st_16cols(lane_base + 32 + 32 * s, w);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint4 b4 = *reinterpret_cast<const uint4*>(st + kSM_XS + 512 * k + lane * 16);
+            w[4 * k] = b4.x; w[4 * k + 1] = b4.y; w[4 * k + 2] = b4.z; w[4 * k + 3] = b4.w;
+          }
+          tmem_st_16cols(lane_base + 32 + 32 * s + 16, w);
+          tmem_st_wait();
+          tc_fence_before();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ready_bar[s]);
+      }
+    }
+    // epilogue: lane quarter q holds features 32 q + lane of the tile
+    const int n = nt * 128 + q * 32 + lane;
+    const float alpha = g.hdr->s_gx * g.hdr->s_gw;
+    const float b = __ldg(g.bias + n);
+    if (__all_sync(0xffffffffu, mbar_wait(&accf_bar, 0, abort_flag))) {
+      tc_fence_after();
+      uint32_t v[16];
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+          "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+            "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+          : "r"(tbase + ((uint32_t)(q * 32) << 16)));
+      tmem_ld_wait();
+      const int M = (int)g.M;
+      if (ks == 1) {
+#pragma unroll
+        for (int m = 0; m < kSM_Tokens; ++m)
+          if (m < M) g.Y[(size_t)m * g.N + n] = bf16_rn(fmaf(alpha, __uint_as_float(v[m]), b));
+      } else {
+        // raw sums -> part[kq]; the warp completing its 32 features adds the parts in K order
+#pragma unroll
+        for (int m = 0; m < kSM_Tokens; ++m)
+          if (m < M) __stcg(g.part + ((size_t)kq * g.M + m) * g.N + n, __uint_as_float(v[m]));
+        __threadfence();
+        __syncwarp();
+        int* cnt = g.cnt + (size_t)nt * 4 + q;
+        int old = 0;
+        if (lane == 0) old = atomicAdd(cnt, 1);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if (old == ks - 1) {
+          __threadfence();
+          for (int m = 0; m < M; ++m) {
+            float t = 0.0f;
+            for (int k = 0; k < ks; ++k) t += __ldcg(g.part + ((size_t)k * g.M + m) * g.N + n);
+            g.Y[(size_t)m * g.N + n] = bf16_rn(fmaf(alpha, t, b));
+          }
+          if (lane == 0) *cnt = 0;   // ready for the next call
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
 // ------------------------------------------------------------ kernel 2, INT4
 // INT4 codes live as E4M3 bytes (exact for -8..7), so each group of 64 is two
 // kind::f8f6f4 MMAs whose fp32 partial sum is an exact integer.  The per-group
@@ -1846,6 +2062,8 @@ svdq_status device_ready() {
       const int i4_smem = dev::kI4Smem;
       d.ok = cudaFuncSetAttribute(dev::gemm_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   dev::kP_Smem) == cudaSuccess &&
+             cudaFuncSetAttribute(dev::gemm_nvfp4_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  dev::kSM_Smem) == cudaSuccess &&
              cudaFuncSetAttribute(dev::gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   i4_smem) == cudaSuccess;
       const int act_smem = dev::kActSmemMax;
@@ -2022,10 +2240,33 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
     CUtensorMap tm_y;
     if (!make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 64, 32))
       return cuda_fail(cudaErrorInvalidValue, "tensor map encode (Y)");
-    const int tiles = (N / 256) * (int)(W.Mp / 256);
-    g.ks = 1;
     g.part = reinterpret_cast<float*>(ws + W.off_part);
     g.cnt = reinterpret_cast<int*>(ws + W.off_cnt);
+    if (M <= dev::kSM_Tokens) {
+      // few tokens: the weight tile as the A operand of a 1-CTA MMA, K split
+      // over idle SMs when the workspace holds the partials
+      const int n_tiles = N / 128;
+      g.ks = 1;
+      if (W.off_cnt > W.off_part)
+        while (g.ks < kMaxKSplit && n_tiles * g.ks * 2 <= num_sms() && g.k_iters % (g.ks * 2) == 0 &&
+               g.k_iters / (g.ks * 2) >= 2)
+          g.ks *= 2;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)(n_tiles * g.ks));
+      cfg.blockDim = dim3(dev::kSM_Threads);
+      cfg.dynamicSmemBytes = dev::kSM_Smem;
+      cfg.stream = stream;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      at[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      const cudaError_t e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_small_kernel, g);
+      if (e != cudaSuccess) return cuda_fail(e, "gemm_nvfp4_small_kernel launch");
+      return launch_status("gemm_nvfp4_small_kernel launch");
+    }
+    const int tiles = (N / 256) * (int)(W.Mp / 256);
+    g.ks = 1;
     if (W.off_cnt > W.off_part) {   // few tokens and tiles: split K over the idle pairs
       while (g.ks < kMaxKSplit && tiles * g.ks * 2 <= num_sms() / 2 && g.k_iters % (g.ks * 2) == 0 &&
              g.k_iters / (g.ks * 2) >= 2)

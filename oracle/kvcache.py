@@ -50,3 +50,30 @@ def decode(q: np.ndarray, s: np.ndarray, z: np.ndarray) -> np.ndarray:
     """(q - z) * s in fp32 (float64 out, holding the fp32 values)."""
     d = (q.astype(np.int32) - z[None, :].astype(np.int32)).astype(F32)
     return (d * np.asarray(s, dtype=F32)[None, :]).astype(F32).astype(np.float64)
+
+
+def attention(Q: np.ndarray, kq, ks, kz, vq, vs, vz, heads: int) -> np.ndarray:
+    """Attention reads over the INT8 cache: for each head h (channels
+    [h d, (h + 1) d), d = C / heads) and query row i,
+        S[i, t] = sum_c Q[i, c] K^[t, c] / sqrt(d),   P = softmax_t(S),
+        O[i, c] = sum_t P[i, t] V^[t, c],
+    with K^ = decode(kq, ks, kz) and V^ = decode(vq, vs, vz) -- the cached
+    keys and values as the codec restores them (exact fp32 values) -- in
+    float64.  Q: Mq x C values (float64 holding fp16/bf16 numbers).
+    Scaled dot-product attention is the VAR transformer's attention; the
+    VAR-Compressor page (INT8 KV缓存量化) stores its cache as INT8, and this is
+    the read of that cache."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = decode(kq, ks, kz)
+    V = decode(vq, vs, vz)
+    Mq, C = Q.shape
+    d = C // heads
+    out = np.empty((Mq, C), dtype=np.float64)
+    for h in range(heads):
+        cols = slice(h * d, (h + 1) * d)
+        S = Q[:, cols] @ K[:, cols].T / np.sqrt(d)
+        S = S - S.max(axis=1, keepdims=True)
+        P = np.exp(S)
+        P = P / P.sum(axis=1, keepdims=True)
+        out[:, cols] = P @ V[:, cols]
+    return out

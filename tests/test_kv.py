@@ -127,3 +127,55 @@ def test_gpu_kv_codec_matches_oracle(gpu, T, C, dtype):
         dec_bytes = T * C + C * 5 + T * C * 2
         print(f"kv {T}x{C} {dtype}: encode {te:.1f} us = {enc_bytes / te / 1e3:.0f} GB/s, "
               f"decode {td:.1f} us = {dec_bytes / td / 1e3:.0f} GB/s (algorithmic bytes)")
+
+
+# ------------------------------------------------------------ attention reads
+def _kv_pair(T, C, seed):
+    kx = skewed_block(T, C, seed)
+    vx = skewed_block(T, C, seed + 1000)
+    return kv.encode(kx) + kv.encode(vx)
+
+
+def test_attention_matches_sdpa_on_decoded_cache():
+    """The oracle's attention equals the library's scaled dot-product
+    attention (torch, float64) over the decoded keys and values, head by head."""
+    import torch
+    T, C, H = 37, 256, 4
+    kq, ks, kz, vq, vs, vz = _kv_pair(T, C, 21)
+    Q = synth.dtype_to_f64(synth.to_dtype(synth.normal(22, "X", 3 * C).reshape(3, C), "fp16"), "fp16")
+    got = kv.attention(Q, kq, ks, kz, vq, vs, vz, H)
+    Kd = torch.from_numpy(kv.decode(kq, ks, kz)); Vd = torch.from_numpy(kv.decode(vq, vs, vz))
+    q = torch.from_numpy(Q)
+    d = C // H
+    for h in range(H):
+        cols = slice(h * d, (h + 1) * d)
+        ref = torch.nn.functional.scaled_dot_product_attention(q[None, None, :, cols], Kd[None, None, :, cols],
+                                                               Vd[None, None, :, cols])[0, 0].numpy()
+        assert np.max(np.abs(got[:, cols] - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_attention_closed_forms():
+    """Zero queries attend uniformly (output = the mean decoded value); a key
+    that dominates every score hands back its own value row; permuting the
+    cached tokens changes nothing; heads do not mix."""
+    T, C, H = 50, 256, 2
+    kq, ks, kz, vq, vs, vz = _kv_pair(T, C, 23)
+    V = kv.decode(vq, vs, vz)
+    out = kv.attention(np.zeros((2, C)), kq, ks, kz, vq, vs, vz, H)
+    assert np.allclose(out, np.broadcast_to(V.mean(axis=0), out.shape), rtol=0, atol=1e-12 * np.abs(V).max())
+    # token 7's key made huge along the query's direction: it takes all the weight
+    Q = np.zeros((1, C)); Q[0, 5] = 1.0; Q[0, 200] = 1.0
+    kq2 = kq.copy(); kq2[:, 5] = kz[5]; kq2[:, 200] = kz[200]            # every key 0 on those channels
+    kq2[7, 5] = 255 if kz[5] < 128 else 0; kq2[7, 200] = 255 if kz[200] < 128 else 0
+    ks2 = ks.copy(); ks2[5] = ks2[200] = np.float32(1e3)
+    o = kv.attention(Q * np.sign(kq2[7:8].astype(int) - kz.astype(int)).clip(-1, 1) + 0.0, kq2, ks2, kz, vq, vs, vz, H)
+    assert np.allclose(o[0, :128], V[7, :128], rtol=0, atol=1e-9 * np.abs(V).max())
+    assert np.allclose(o[0, 128:], V[7, 128:], rtol=0, atol=1e-9 * np.abs(V).max())
+    perm = np.random.default_rng(0).permutation(T)
+    Qr = synth.dtype_to_f64(synth.to_dtype(synth.normal(24, "X", 2 * C).reshape(2, C), "fp16"), "fp16")
+    a = kv.attention(Qr, kq, ks, kz, vq, vs, vz, H)
+    b = kv.attention(Qr, kq[perm], ks, kz, vq[perm], vs, vz, H)
+    assert np.allclose(a, b, rtol=0, atol=1e-12 * np.abs(a).max())
+    Qh = Qr.copy(); Qh[:, 128:] *= 3.0                                  # head 1's queries only
+    c = kv.attention(Qh, kq, ks, kz, vq, vs, vz, H)
+    assert np.array_equal(c[:, :128], a[:, :128])

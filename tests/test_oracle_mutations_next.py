@@ -28,6 +28,7 @@ KV_PINS = [TK.test_golden_codes, TK.test_round_trip_error_is_half_a_step, TK.tes
            TK.test_asymmetric_beats_symmetric_on_skewed_data]
 LORA_PINS = [lambda: TL.test_oracle_lora_adds_exactly_xab_without_smoothing("nvfp4"),
              lambda: TL.test_oracle_lora_with_smoothing_matches_xab_to_the_dtype("int4", "fp16")]
+ATT_PINS = [TK.test_attention_matches_sdpa_on_decoded_cache, TK.test_attention_closed_forms]
 SHARD_PINS = [lambda: TS.test_oracle_shard_is_the_full_layers_columns("int4", "fp16"),
               lambda: TS.test_oracle_shard_is_the_full_layers_columns("nvfp4", "bf16")]
 
@@ -83,6 +84,25 @@ def _shard_l2_unshifted(p, n0, n1):
                        p.R[:, n0:n1], wq, p.s_gx, p.bias[n0:n1])
 
 
+def _attention_variant(scale_all=False, softmax_axis=1, heads_mix=False):
+    def attention(Q, kq, ks, kz, vq, vs, vz, heads):
+        Q = np.asarray(Q, dtype=np.float64)
+        K = kv.decode(kq, ks, kz); V = kv.decode(vq, vs, vz)
+        Mq, C = Q.shape
+        d = C // heads
+        out = np.empty((Mq, C))
+        for h in range(heads):
+            cols = slice(h * d, (h + 1) * d)
+            qc = Q if heads_mix else Q[:, cols]
+            kc = K if heads_mix else K[:, cols]
+            S = qc @ kc.T / np.sqrt(C if scale_all else d)
+            S = S - S.max(axis=softmax_axis, keepdims=True)
+            P = np.exp(S); P = P / P.sum(axis=softmax_axis, keepdims=True)
+            out[:, cols] = P @ V[:, cols]
+        return out
+    return attention
+
+
 MUTATIONS = {
     "kv_divisor_256": (kv, "channel_params", _params(divisor=256.0), KV_PINS),
     "kv_zero_point_sign": (kv, "channel_params", _params(zsign=1.0), KV_PINS),
@@ -93,6 +113,9 @@ MUTATIONS = {
     "lora_lambda_divides": (sq, "append_lora", _lora_lambda_divides, LORA_PINS),
     "shard_bias_unshifted": (sq, "shard_columns", _shard_bias_unshifted, SHARD_PINS),
     "shard_l2_unshifted": (sq, "shard_columns", _shard_l2_unshifted, SHARD_PINS),
+    "attention_scaled_by_all_channels": (kv, "attention", _attention_variant(scale_all=True), ATT_PINS),
+    "attention_softmax_over_queries": (kv, "attention", _attention_variant(softmax_axis=0), ATT_PINS),
+    "attention_heads_mixed": (kv, "attention", _attention_variant(heads_mix=True), ATT_PINS),
 }
 
 
@@ -104,4 +127,4 @@ def test_planted_mistake_is_caught(name, monkeypatch):
 
 
 def test_unmutated_pins_pass():
-    assert _run(KV_PINS + LORA_PINS + SHARD_PINS) == 0
+    assert _run(KV_PINS + LORA_PINS + SHARD_PINS + ATT_PINS) == 0

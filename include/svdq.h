@@ -191,6 +191,29 @@ svdq_status svdq_kv_encode(const void* X, int64_t T, int32_t C, int32_t dtype, u
 svdq_status svdq_kv_decode(const uint8_t* codes, const float* scale, const uint8_t* zero, int64_t T, int32_t C,
                            int32_t dtype, void* Y, svdq_stream stream);
 
+/*
+ * Attention reads over INT8 caches (the read side of the codec above): scaled
+ * dot-product attention of Mq query rows against T cached keys and values
+ * held as codes, per head, without materialising the decoded cache:
+ *   for head h (channels [h d, (h + 1) d), d = C / heads),
+ *   S[i,t] = sum_c Q[i,c] K^[t,c] / sqrt(d),  P = softmax over t,
+ *   out[i,c] = sum_t P[i,t] V^[t,c],   K^ = (kcodes - kzero) kscale, V^ likewise
+ * (the decoded values in fp32).  Q: Mq x C, dtype (SVDQ_BF16 / SVDQ_F16);
+ * kcodes, vcodes: T x C uint8; kscale, vscale: C fp32; kzero, vzero: C uint8
+ * (as svdq_kv_encode writes them); out: Mq x C fp32.  All device pointers,
+ * 16-byte aligned, owned by the caller; workspace >= the bytes below.
+ * 1 <= Mq <= 16, T >= 1, d = 64 or 128 (else SVDQ_ERR_UNSUPPORTED).
+ * Asynchronous on `stream` (two kernels: 256-token chunks, then a combine in
+ * chunk order, so results are reproducible bit for bit).  Errors:
+ * SVDQ_ERR_INVALID_ARG, SVDQ_ERR_WORKSPACE, SVDQ_ERR_ALIGNMENT,
+ * SVDQ_ERR_UNSUPPORTED, SVDQ_ERR_CUDA.
+ */
+size_t svdq_kv_attention_workspace_bytes(int64_t T, int32_t C, int32_t heads, int32_t Mq);
+svdq_status svdq_kv_attention(const void* Q, int32_t Mq, const uint8_t* kcodes, const float* kscale,
+                              const uint8_t* kzero, const uint8_t* vcodes, const float* vscale, const uint8_t* vzero,
+                              int64_t T, int32_t C, int32_t heads, int32_t dtype, float* out, void* workspace,
+                              size_t ws_bytes, svdq_stream stream);
+
 /* Device workspace bytes svdq_linear needs for M tokens. */
 size_t svdq_workspace_bytes(const svdq_params* p, int64_t M);
 

@@ -57,6 +57,9 @@ def _load():
         "svdq_kv_workspace_bytes": (sz, [i64, ctypes.c_int32]),
         "svdq_kv_encode": (ctypes.c_int, [vp, i64, ctypes.c_int32, ctypes.c_int32, vp, vp, vp, vp, sz, vp]),
         "svdq_kv_decode": (ctypes.c_int, [vp, vp, vp, i64, ctypes.c_int32, ctypes.c_int32, vp, vp]),
+        "svdq_kv_attention_workspace_bytes": (sz, [i64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]),
+        "svdq_kv_attention": (ctypes.c_int, [vp, ctypes.c_int32, vp, vp, vp, vp, vp, vp, i64, ctypes.c_int32,
+                                             ctypes.c_int32, ctypes.c_int32, vp, vp, sz, vp]),
         "svdq_workspace_bytes": (sz, [P, i64]),
         "svdq_linear": (ctypes.c_int, [P, vp, vp, i64, vp, vp, sz, vp]),
         "svdq_quantize_act": (ctypes.c_int, [P, vp, vp, i64, vp, sz, vp]),
@@ -82,7 +85,7 @@ EXPORTED = ("svdq_blob_bytes", "svdq_prepare", "svdq_blob_check", "svdq_blob_exp
             "svdq_workspace_bytes", "svdq_linear", "svdq_quantize_act", "svdq_gemm", "svdq_export_act", "svdq_get_status",
             "svdq_status_string", "svdq_last_error_string", "svdq_probe_cvt", "svdq_probe_div", "svdq_probe_tc",
             "svdq_linear_noalloc", "svdq_probe_timeout", "svdq_kv_workspace_bytes", "svdq_kv_encode",
-            "svdq_kv_decode")
+            "svdq_kv_decode", "svdq_kv_attention_workspace_bytes", "svdq_kv_attention")
 NOALLOC_SCRATCH_BYTES = 16 << 20   # SVDQ_NOALLOC_SCRATCH_BYTES
 
 
@@ -247,6 +250,19 @@ def kv_encode(X, T: int, C: int, dtype: str, codes, scale, zero, workspace, stre
 def kv_decode(codes, scale, zero, T: int, C: int, dtype: str, Y, stream=None):
     st = _lib.svdq_kv_decode(_ptr(codes), _ptr(scale), _ptr(zero), T, C, DTYPE[dtype], _ptr(Y), _stream(stream))
     _check(st, "svdq_kv_decode")
+
+
+def kv_attention_workspace_bytes(T: int, C: int, heads: int, Mq: int) -> int:
+    return _lib.svdq_kv_attention_workspace_bytes(T, C, heads, Mq)
+
+
+def kv_attention(Q, Mq: int, kcodes, kscale, kzero, vcodes, vscale, vzero, T: int, C: int, heads: int, dtype: str,
+                 out, workspace, stream=None):
+    """Attention of Mq query rows over INT8-coded keys and values (device tensors); out: Mq x C fp32."""
+    st = _lib.svdq_kv_attention(_ptr(Q), Mq, _ptr(kcodes), _ptr(kscale), _ptr(kzero), _ptr(vcodes), _ptr(vscale),
+                                _ptr(vzero), T, C, heads, DTYPE[dtype], _ptr(out), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "svdq_kv_attention")
 
 
 def linear_noalloc(p: svdq_params, blob_dev, X, M: int, Y, stream=None):

@@ -179,3 +179,67 @@ def test_attention_closed_forms():
     Qh = Qr.copy(); Qh[:, 128:] *= 3.0                                  # head 1's queries only
     c = kv.attention(Qh, kq, ks, kz, vq, vs, vz, H)
     assert np.array_equal(c[:, :128], a[:, :128])
+
+
+def test_attention_argument_checks():
+    import rank_gemm_svdq_b200 as sv
+    assert sv.kv_attention_workspace_bytes(300, 512, 4, 3) == 4 * 2 * 3 * (128 + 2) * 4
+    assert sv.kv_attention_workspace_bytes(0, 512, 4, 3) == 0
+    assert sv.kv_attention_workspace_bytes(10, 500, 3, 1) == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("T,C,H,Mq,dtype", [(1, 256, 4, 1, "bf16"), (300, 512, 4, 3, "fp16"),
+                                            (257, 1024, 16, 16, "bf16"), (4096, 4096, 32, 1, "bf16"),
+                                            (4096, 4096, 32, 8, "bf16")])
+def test_gpu_attention_reads_match_oracle(gpu, T, C, H, Mq, dtype):
+    """svdq_kv_attention over codes written by svdq_kv_encode against the
+    oracle's attention over the decoded cache (fp32 output, relative
+    Frobenius error <= 1e-5 and per-element <= 1e-4 of the output range);
+    two calls give identical bits.  The 4096-token VAR-like cache is timed."""
+    import torch
+    import rank_gemm_svdq_b200 as sv
+    from oracle import svdquant as sq
+    kbits, kx = _block_bits(T, C, dtype, seed=T + C + 1)
+    vbits, vx = _block_bits(T, C, dtype, seed=T + C + 2)
+    qx = synth.normal(T + Mq, "X", Mq * C).reshape(Mq, C)
+    qbits = synth.to_dtype(qx, dtype)
+    qbits = qbits.view(np.uint16) if dtype == "fp16" else qbits
+    Q = synth.dtype_to_f64(synth.to_dtype(qx, dtype), dtype)
+    dev = {}
+    for name, bits in (("k", kbits), ("v", vbits)):
+        X = torch.from_numpy(bits.view(np.int16)).cuda()
+        codes = torch.empty((T, C), dtype=torch.uint8, device="cuda")
+        scale = torch.empty(C, dtype=torch.float32, device="cuda")
+        zero = torch.empty(C, dtype=torch.uint8, device="cuda")
+        ws = torch.empty(sv.kv_workspace_bytes(T, C), dtype=torch.uint8, device="cuda")
+        sv.kv_encode(X, T, C, dtype, codes, scale, zero, ws)
+        dev[name] = (codes, scale, zero)
+    Qd = torch.from_numpy(qbits.view(np.int16)).cuda()
+    out = torch.empty((Mq, C), dtype=torch.float32, device="cuda")
+    wsa = torch.empty(sv.kv_attention_workspace_bytes(T, C, H, Mq), dtype=torch.uint8, device="cuda")
+    sv.kv_attention(Qd, Mq, *dev["k"], *dev["v"], T, C, H, dtype, out, wsa)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy().astype(np.float64)
+    kq, ks, kz = kv.encode(kx)
+    vq, vs, vz = kv.encode(vx)
+    assert np.array_equal(dev["k"][0].cpu().numpy(), kq) and np.array_equal(dev["v"][0].cpu().numpy(), vq)
+    ref = kv.attention(Q, kq, ks, kz, vq, vs, vz, H)
+    assert sq.rel_fro(got, ref) <= 1e-5, sq.rel_fro(got, ref)
+    assert np.max(np.abs(got - ref)) <= 1e-4 * np.max(np.abs(ref))
+    out2 = torch.empty_like(out)
+    sv.kv_attention(Qd, Mq, *dev["k"], *dev["v"], T, C, H, dtype, out2, wsa)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+    if T * C >= 1 << 24:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        ts = []
+        for i in range(12):
+            flush.fill_(i)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(); sv.kv_attention(Qd, Mq, *dev["k"], *dev["v"], T, C, H, dtype, out, wsa); b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3)
+        t = float(np.median(ts[2:]))
+        byts = 2 * T * C + Mq * C * 2 + Mq * C * 4 + 10 * C
+        print(f"kv attention {T}x{C} heads {H} queries {Mq}: {t:.1f} us = {byts / t / 1e3:.0f} GB/s (algorithmic bytes)")

@@ -244,6 +244,21 @@ def forward_bf16(x: np.ndarray, p: Prepared, group: int = 64) -> np.ndarray:
     return formats.to_bf16(forward(x, p, group))
 
 
+def next_layer_input(x: np.ndarray, p: Prepared, p_next: Prepared, group: int = 64) -> ActQ:
+    """The quantised input of the next layer when this layer feeds it.
+
+    The next layer reads this layer's output as the layer writes it (bf16 Y)
+    and treats it like any activation: its own smoothing, dynamic
+    quantisation and low-rank down projection, i.e. quantize_act(bf16(Y),
+    p_next).  Fusing this into this layer's epilogue only moves where it is
+    computed ("DeepCompressor…" SVDQuant section: the low-rank branch is
+    folded into the low-bit kernel to save the activation round trip; the
+    same saving at the boundary between two layers).
+    """
+    y = forward_bf16(x, p, group)
+    return quantize_act(y, p_next, group)
+
+
 def exact_output(x: np.ndarray, Wt: np.ndarray, bias) -> np.ndarray:
     """The unquantised layer X W + b in float64 (for error reports)."""
     b = 0.0 if bias is None else np.asarray(bias, dtype=np.float64)[None, :]

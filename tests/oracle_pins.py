@@ -491,3 +491,91 @@ def pin_lapack_factors_match_jacobi(sq):
         assert np.linalg.norm(P - Q) <= 4 * u * np.linalg.norm(P)
         ra = np.linalg.norm(W_hat - P); rb = np.linalg.norm(W_hat - Q)
         assert abs(ra - rb) <= 4 * u * np.linalg.norm(P)
+
+
+# ---------------------------------------------------------------- chained layers
+def _bf16_exact(q: Fraction) -> float:
+    """An exact rational rounded to the nearest bf16 value (8 significant bits),
+    ties to the even significand (normal range only)."""
+    if q == 0:
+        return 0.0
+    sign = -1 if q < 0 else 1
+    a = abs(q)
+    e = math.frexp(float(a))[1] - 1                 # 2^e <= a < 2^(e+1), fixed up exactly below
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    ulp = Fraction(2) ** (e - 7)
+    n = a / ulp
+    k = n.numerator // n.denominator
+    rem = n - k
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and k % 2 == 1):
+        k += 1
+    return sign * float(k * ulp)
+
+
+def _nearest_code(t: float, values, max_code: int) -> int:
+    """Exhaustive nearest non-negative code to |t| among codes 0..max_code,
+    ties to the even code, magnitudes past the largest clamped to it."""
+    a = abs(t)
+    best, best_err = 0, None
+    for c in range(max_code + 1):
+        err = abs(Fraction(a) - Fraction(float(values[c])))
+        if best_err is None or err < best_err or (err == best_err and c % 2 == 0):
+            best, best_err = c, err
+    return best
+
+
+def pin_next_layer_input_bruteforce(sq):
+    """The next layer's quantised input, by brute force on a tiny pair of
+    NVFP4 layers: this layer's Y in exact rationals from its (pinned) codes,
+    rounded to bf16 by exact arithmetic, smoothed by the NEXT layer's
+    1/lambda in fp32, block scales and codes by exhaustive nearest search
+    over the E4M3 / E2M1 grids under the next layer's tensor scale, and u'
+    exact from the bf16-rounded smoothed values and the next layer's L1."""
+    from oracle import formats
+    rng = np.random.default_rng(31)
+    M, K, N, N2, r = 3, 16, 32, 16, 2
+    x = rng.standard_normal((M, K)); x[:, 3] *= 20
+    x = formats.to_bf16(x)
+    Wt1 = rng.standard_normal((N, K)).astype(np.float32); b1 = rng.standard_normal(N).astype(np.float32)
+    Wt2 = (rng.standard_normal((N2, N)) * 0.2).astype(np.float32); b2 = rng.standard_normal(N2).astype(np.float32)
+    p1 = sq.prepare(x, Wt1, b1, r, "nvfp4", "bf16")
+    y_cal = sq.forward_bf16(x, p1)                  # the next layer is calibrated on what it sees
+    y_cal[:, ::5] *= 3.0                            # ... widened so that its outliers differ from Y's
+    p2 = sq.prepare(formats.to_bf16(y_cal), Wt2, b2, r, "nvfp4", "bf16")
+    a = sq.next_layer_input(x, p1, p2)
+    _, a1, _, _ = sq.forward(x, p1, return_parts=True)
+    sgx1, sgw1 = Fraction(float(p1.s_gx)), Fraction(float(p1.wq.s_g))
+    dx = [[sgx1 * Fraction(float(formats.E4M3_VALUES[a1.scales[m, k // 16]]))
+           * Fraction(float(formats.E2M1_VALUES[a1.codes[m, k]])) for k in range(K)] for m in range(M)]
+    dw = [[sgw1 * Fraction(float(formats.E4M3_VALUES[p1.wq.scales[n, k // 16]]))
+           * Fraction(float(formats.E2M1_VALUES[p1.wq.codes[n, k]])) for k in range(K)] for n in range(N)]
+    x16 = [[Fraction(_bf16_exact(Fraction(float(np.float32(x[m, k]) * np.float32(p1.inv_lambda[k])))))
+            for k in range(K)] for m in range(M)]
+    s_g2 = np.float32(p2.s_gx)
+    six = np.float32(np.float32(6.0) * s_g2)
+    for m in range(M):
+        u1 = [sum(x16[m][k] * Fraction(float(p1.L1[k, i])) for k in range(K)) for i in range(r)]
+        y = [_bf16_exact(sum(dx[m][k] * dw[n][k] for k in range(K))
+                         + sum(u1[i] * Fraction(float(p1.L2[i, n])) for i in range(r)) + Fraction(float(b1[n])))
+             for n in range(N)]
+        xh = [np.float32(y[n]) * np.float32(p2.inv_lambda[n]) for n in range(N)]
+        for blk in range(N // 16):
+            vals = xh[16 * blk:16 * blk + 16]
+            amax = max(abs(float(v)) for v in vals)
+            ratio = np.float32(np.float32(amax) / six)
+            e = _nearest_code(float(ratio), formats.E4M3_VALUES, 0x7E)
+            assert a.scales[m, blk] == e, (m, blk, a.scales[m, blk], e)
+            d = np.float32(np.float32(formats.E4M3_VALUES[e]) * s_g2)
+            for j, v in enumerate(vals):
+                if d == 0:
+                    code = 0
+                else:
+                    t = np.float32(v / d)
+                    code = _nearest_code(float(t), formats.E2M1_VALUES, 7) | (8 if math.copysign(1.0, float(t)) < 0 else 0)
+                assert a.codes[m, 16 * blk + j] == code, (m, blk, j, a.codes[m, 16 * blk + j], code)
+        for i in range(r):
+            u = sum(Fraction(_bf16_exact(Fraction(float(xh[n])))) * Fraction(float(p2.L1[n, i])) for n in range(N))
+            assert abs(a.u[m, i] - float(u)) <= 1e-12 * (abs(float(u)) + 1), (m, i, a.u[m, i], float(u))

@@ -1,12 +1,16 @@
-"""Planted mistakes in the oracle's next-row functions (KV-cache codec, LoRA
-append, column shards) must each fail at least one of their pins (the CPU
-tests of tests/test_kv.py, tests/test_lora.py and tests/test_shard.py)."""
+"""Planted mistakes in the oracle's next-row functions (KV-cache codec and
+attention reads, LoRA append, column shards, the chained next-layer input)
+must each fail at least one of their pins (the CPU tests of tests/test_kv.py,
+tests/test_lora.py, tests/test_shard.py and the brute-force chain pin)."""
+import dataclasses
+
 import numpy as np
 import pytest
 
 import oracle.formats as formats
 import oracle.kvcache as kv
 import oracle.svdquant as sq
+from tests import oracle_pins as P
 from tests import test_kv as TK
 from tests import test_lora as TL
 from tests import test_shard as TS
@@ -103,7 +107,27 @@ def _attention_variant(scale_all=False, softmax_axis=1, heads_mix=False):
     return attention
 
 
+CHAIN_PINS = [lambda: P.pin_next_layer_input_bruteforce(sq)]
+
+
+def _next_input_unrounded_y(x, p, p_next, group=64):
+    return sq.quantize_act(sq.forward(x, p, group), p_next, group)
+
+
+def _next_input_unsmoothed(x, p, p_next, group=64):
+    q = dataclasses.replace(p_next, inv_lambda=np.ones_like(p_next.inv_lambda))
+    return sq.quantize_act(sq.forward_bf16(x, p, group), q, group)
+
+
+def _next_input_this_layers_tensor_scale(x, p, p_next, group=64):
+    q = dataclasses.replace(p_next, s_gx=p.s_gx)
+    return sq.quantize_act(sq.forward_bf16(x, p, group), q, group)
+
+
 MUTATIONS = {
+    "chain_y_not_rounded_to_bf16": (sq, "next_layer_input", _next_input_unrounded_y, CHAIN_PINS),
+    "chain_next_smoothing_dropped": (sq, "next_layer_input", _next_input_unsmoothed, CHAIN_PINS),
+    "chain_tensor_scale_of_this_layer": (sq, "next_layer_input", _next_input_this_layers_tensor_scale, CHAIN_PINS),
     "kv_divisor_256": (kv, "channel_params", _params(divisor=256.0), KV_PINS),
     "kv_zero_point_sign": (kv, "channel_params", _params(zsign=1.0), KV_PINS),
     "kv_range_not_widened": (kv, "channel_params", _params(widen=False), KV_PINS),
@@ -127,4 +151,4 @@ def test_planted_mistake_is_caught(name, monkeypatch):
 
 
 def test_unmutated_pins_pass():
-    assert _run(KV_PINS + LORA_PINS + SHARD_PINS + ATT_PINS) == 0
+    assert _run(KV_PINS + LORA_PINS + SHARD_PINS + ATT_PINS + CHAIN_PINS) == 0

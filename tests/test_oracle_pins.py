@@ -87,3 +87,7 @@ def test_act_tensor_scale_in_prepare():
 
 def test_lapack_factors_match_jacobi():
     P.pin_lapack_factors_match_jacobi(svdquant)
+
+
+def test_next_layer_input_bruteforce():
+    P.pin_next_layer_input_bruteforce(svdquant)

@@ -448,6 +448,83 @@ def error_report(args):
                           "seconds": time.perf_counter() - t0}), flush=True)
 
 
+def run_chain(args):
+    """Two chained layers, FLUX FFN up (M 4608, K 3072 -> N 12288) into an FFN
+    down projection (12288 -> 3072, rank 32), both NVFP4: the up projection's
+    GEMM emits the down projection's quantised input (svdq_gemm_chain) against
+    the same two layers run one after the other (svdq_linear twice, the
+    12288-wide bf16 output written and read back).  One step = both layers
+    after a 256 MiB flush; prints one JSON line (TFLOP/s over both layers)."""
+    import torch
+    import rank_gemm_svdq_b200 as sv
+    import synth
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    wl = synth.make_workload(WORKLOAD, seed=0)
+    M, K, N, r = wl.M, wl.K, wl.N, wl.rank
+    N2, r2 = 3072, 32
+    p1 = sv.params(K, N, r, "nvfp4", "bf16", wl.alpha, wl.smooth)
+    blob1 = torch.from_numpy(sv.prepare(p1, wl.Wt, wl.bias, wl.X)[0]).to(dev)
+    X = torch.from_numpy(wl.X.view(np.int16)).to(dev).view(torch.bfloat16)
+    ws1 = torch.empty(sv.workspace_bytes(p1, M), dtype=torch.uint8, device=dev)
+    Y1 = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    sv.linear(p1, blob1, X, M, Y1, ws1)
+    torch.cuda.synchronize()
+    # the down projection is calibrated on what it sees: the up projection's output
+    p2 = sv.params(N, N2, r2, "nvfp4", "bf16")
+    Wt2, b2 = synth.make_weight(1, N2, N), synth.make_bias(1, N2)
+    blob2 = torch.from_numpy(sv.prepare(p2, Wt2, b2, Y1.view(torch.int16).cpu().numpy())[0]).to(dev)
+    ws = torch.empty(sv.chain_workspace_bytes(p1, p2, M), dtype=torch.uint8, device=dev)
+    ws2 = torch.empty(sv.workspace_bytes(p2, M), dtype=torch.uint8, device=dev)
+    Y2 = torch.empty((M, N2), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def chained(i):
+        sv.quantize_act(p1, blob1, X, M, ws, stream)
+        sv.gemm_chain(p1, blob1, M, p2, blob2, ws, ws2, stream)
+        sv.gemm(p2, blob2, M, Y2, ws2, stream)
+
+    def unfused(i):
+        sv.linear(p1, blob1, X, M, Y1, ws1, stream)
+        sv.linear(p2, blob2, Y1, M, Y2, ws2, stream)
+
+    def timed(fn, steps):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        with torch.cuda.stream(stream):
+            for i in range(steps):
+                flush.fill_(i & 0xFF)
+                evs[i][0].record(stream)
+                fn(i)
+                evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        return float(np.median([a.elapsed_time(b) for a, b in evs]))
+
+    for fn in (chained, unfused):
+        timed(fn, args.warmup)
+    assert sv.get_status() == sv.OK
+    sampler = ClockSampler(device_smi_id(torch, dev.index or 0))
+    sampler.start()
+    time.sleep(0.3)
+    t0 = time.time()
+    ms_c = timed(chained, args.steps)
+    ms_u = timed(unfused, args.steps)
+    t1 = time.time()
+    sampler.stop()
+    st = sv.get_status()
+    assert st == sv.OK, sv.status_string(st)
+    fl = flops(M, K, N, r) + flops(M, N, N2, r2)
+    print(json.dumps({
+        "metric": METRIC, "value": fl / (ms_c * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_c, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+        "config": {"workload": f"{WORKLOAD} -> ffn down {N}x{N2} r{r2}, chained", "M": M,
+                   "layers": [[K, N, r], [N, N2, r2]], "l2": "256 MiB flush per step"},
+        "unfused": {"ms_per_step": ms_u, "value": fl / (ms_u * 1e-3) / 1e12},
+        "clocks": sampler.summary(t0, t1), "gpu_launches": 8 * args.steps}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -461,8 +538,13 @@ def main():
                     help="run on the first M tokens of the workload (calibration still uses all of them)")
     ap.add_argument("--error-report", default="",
                     help="with --impl reference: 'all' or comma-separated presets; prints E_0 / E_r")
+    ap.add_argument("--chain", action="store_true",
+                    help="two chained NVFP4 layers (FFN up -> down), fused next-layer input vs unfused")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.chain:
+        run_chain(args)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -249,6 +249,41 @@ svdq_status svdq_gemm(const svdq_params* p, const void* blob_dev, int64_t M, voi
                       size_t ws_bytes, svdq_stream stream);
 
 /*
+ * Chained layers: this layer's GEMM emits the NEXT layer's quantised input,
+ * so this layer's output never makes a bf16 round trip through HBM (the
+ * fusion argument of the "DeepCompressor…" SVDQuant section, where the
+ * low-rank branch rides in the low-bit kernel to save activation traffic,
+ * carried to the boundary between two layers).  The next layer's input is
+ * this layer's bf16 output y; its quantised form is what the next layer's
+ * activation kernel would make of y: x^' = fp32(y) * inv_lambda', NVFP4
+ * codes and E4M3 block scales under the next layer's static tensor scale,
+ * and u' = X^'16 L1' with X^'16 = bf16(x^').
+ * Call it where svdq_gemm would be called: `workspace` holds this layer's
+ * quantised input (from svdq_quantize_act, or from a previous chained call
+ * as its ws_next).  On return (stream order) ws_next holds the next layer's
+ * quantised input exactly as svdq_quantize_act(p_next, blob_next, y, M,
+ * ws_next) leaves it, codes and scales bit for bit; u' equal up to fp32
+ * summation order (per output tile, then across tiles in order).  Finish
+ * with svdq_gemm(p_next, blob_next, M, Y', ws_next) or chain again.
+ *   Both layers NVFP4; p_next->K == p->N; p_next->act_dtype == SVDQ_BF16;
+ *   p_next->rank 0, 16 or 32 (else SVDQ_ERR_UNSUPPORTED / INVALID_ARG).
+ *   workspace >= svdq_chain_workspace_bytes(p, p_next, M) (this layer's
+ *   workspace plus the next layer's partial down projections, one per
+ *   256-column output tile, fp32); ws_next >= svdq_workspace_bytes(p_next, M).
+ *   Above 128 tokens this is one GEMM launch whose epilogue quantises and
+ *   runs the partial down projection on the tensor cores, plus a small
+ *   kernel that adds the partials; up to 128 tokens (this layer's output at
+ *   most 128 rows) the GEMM writes y into the workspace and the next
+ *   layer's activation kernel reads it.
+ * All pointers device, 16-byte aligned, owned by the caller.  Asynchronous on
+ * `stream`; errors as svdq_gemm.
+ */
+size_t svdq_chain_workspace_bytes(const svdq_params* p, const svdq_params* p_next, int64_t M);
+svdq_status svdq_gemm_chain(const svdq_params* p, const void* blob_dev, int64_t M, const svdq_params* p_next,
+                            const void* blob_next_dev, void* workspace, size_t ws_bytes, void* ws_next,
+                            size_t ws_next_bytes, svdq_stream stream);
+
+/*
  * After svdq_linear: copy the quantised activations out of the workspace in
  * canonical form (synchronises `stream`).  Any output pointer may be NULL.
  *   codes   M x K host, one code per byte (INT4 int8 / NVFP4 E2M1 low nibble)

@@ -64,6 +64,8 @@ def _load():
         "svdq_linear": (ctypes.c_int, [P, vp, vp, i64, vp, vp, sz, vp]),
         "svdq_quantize_act": (ctypes.c_int, [P, vp, vp, i64, vp, sz, vp]),
         "svdq_gemm": (ctypes.c_int, [P, vp, i64, vp, vp, sz, vp]),
+        "svdq_chain_workspace_bytes": (sz, [P, P, i64]),
+        "svdq_gemm_chain": (ctypes.c_int, [P, vp, i64, P, vp, vp, sz, vp, sz, vp]),
         "svdq_export_act": (ctypes.c_int, [P, vp, i64, vp, vp, vp, vp]),
         "svdq_get_status": (ctypes.c_int, [vp]),
         "svdq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -85,7 +87,8 @@ EXPORTED = ("svdq_blob_bytes", "svdq_prepare", "svdq_blob_check", "svdq_blob_exp
             "svdq_workspace_bytes", "svdq_linear", "svdq_quantize_act", "svdq_gemm", "svdq_export_act", "svdq_get_status",
             "svdq_status_string", "svdq_last_error_string", "svdq_probe_cvt", "svdq_probe_div", "svdq_probe_tc",
             "svdq_linear_noalloc", "svdq_probe_timeout", "svdq_kv_workspace_bytes", "svdq_kv_encode",
-            "svdq_kv_decode", "svdq_kv_attention_workspace_bytes", "svdq_kv_attention")
+            "svdq_kv_decode", "svdq_kv_attention_workspace_bytes", "svdq_kv_attention",
+            "svdq_chain_workspace_bytes", "svdq_gemm_chain")
 NOALLOC_SCRATCH_BYTES = 16 << 20   # SVDQ_NOALLOC_SCRATCH_BYTES
 
 
@@ -285,6 +288,20 @@ def gemm(p: svdq_params, blob_dev, M: int, Y, workspace, stream=None):
     """Kernel 2 only: workspace -> Y (after quantize_act on the same stream)."""
     _check(_lib.svdq_gemm(ctypes.byref(p), _ptr(blob_dev), M, _ptr(Y), _ptr(workspace),
                           workspace.numel() * workspace.element_size(), _stream(stream)), "svdq_gemm")
+
+
+def chain_workspace_bytes(p: svdq_params, p_next: svdq_params, M: int) -> int:
+    """Workspace bytes of gemm_chain (0 if the pair of layers cannot chain)."""
+    return _lib.svdq_chain_workspace_bytes(ctypes.byref(p), ctypes.byref(p_next), M)
+
+
+def gemm_chain(p: svdq_params, blob_dev, M: int, p_next: svdq_params, blob_next_dev, workspace, ws_next,
+               stream=None):
+    """This layer's GEMM emitting the next layer's quantised input into ws_next
+    (in place of quantize_act(p_next, ..., Y, ...)); finish with gemm(p_next, ...)."""
+    _check(_lib.svdq_gemm_chain(ctypes.byref(p), _ptr(blob_dev), M, ctypes.byref(p_next), _ptr(blob_next_dev),
+                                _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(ws_next),
+                                ws_next.numel() * ws_next.element_size(), _stream(stream)), "svdq_gemm_chain")
 
 
 def export_act(p: svdq_params, workspace, M: int, stream=None):

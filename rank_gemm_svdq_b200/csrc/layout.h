@@ -138,6 +138,22 @@ SVDQ_HD inline int act_nv_ks(int64_t Mp, int K) {
   return ks;
 }
 
+// NVFP4 up to 256 tokens (the 32-token activation kernel): with few live
+// 32-token groups, ks CTAs split a group's K range (a power of two dividing
+// K / 256, at most kActGMaxKs).  Up to 8 they form a cluster and add their
+// partial down projections through distributed shared memory; above 8 the
+// partials meet in the workspace ([groups][ks][32][r] fp32 plus one 64-bit
+// arrival word per group, tagged per call like the 128-token kernel's).
+constexpr int kActGMaxKs = 32;
+constexpr int kActClusterKs = 8;
+SVDQ_HD inline int act_small_ks(int64_t M, int K) {
+  const int64_t groups = (M + 31) / 32;
+  const int chunks = K / 256;
+  int ks = 1;
+  while (ks < kActGMaxKs && groups * ks * 2 <= kActSizingSMs && chunks % (ks * 2) == 0) ks *= 2;
+  return ks;
+}
+
 inline WsLayout ws_layout(const svdq_params& p, int64_t M) {
   WsLayout L{};
   const size_t K = (size_t)p.K;
@@ -166,8 +182,48 @@ inline WsLayout ws_layout(const svdq_params& p, int64_t M) {
       L.off_ucnt = off;
       off = align_up(off + (Mp / 128) * 8);
     }
+  } else if (p.fmt == SVDQ_NVFP4 && M >= 1) {   // the 32-token kernel with its K split in the workspace
+    const int ks = act_small_ks(M, p.K);
+    if (ks > kActClusterKs && p.rank > 0) {
+      const size_t groups = (size_t)((M + 31) / 32);
+      off = align_up(off + groups * (size_t)ks * 32 * (size_t)p.rank * 4);
+      L.off_ucnt = off;
+      off = align_up(off + groups * 8);
+    }
   }
   L.total = off > 0 ? off : kAlign;
+  return L;
+}
+
+// NVFP4 up to this many tokens: the GEMM streams each weight tile as the A
+// operand of a 1-CTA MMA with the tokens as a narrow B operand.
+constexpr int64_t kFewTokens = 128;
+
+// Chained layers (svdq_gemm_chain): this layer's GEMM emits the next layer's
+// quantised input.  Both NVFP4, the next layer's input bf16 (this layer's
+// output type) and its rank 0, 16 or 32.
+inline svdq_status chain_supported(const svdq_params& p, const svdq_params& pn) {
+  if (p.fmt != SVDQ_NVFP4 || pn.fmt != SVDQ_NVFP4 || pn.act_dtype != SVDQ_BF16) return SVDQ_ERR_UNSUPPORTED;
+  if (pn.K != p.N) return SVDQ_ERR_INVALID_ARG;
+  if (pn.rank != 0 && pn.rank != 16 && pn.rank != 32) return SVDQ_ERR_UNSUPPORTED;
+  return SVDQ_OK;
+}
+
+// Workspace of a chained call: this layer's workspace, then above kFewTokens
+// the partial down projections of the next layer, [N/256][Mp][r'] fp32 (one
+// per output tile column), or up to kFewTokens an M x N bf16 buffer for this
+// layer's output (there the call runs the GEMM and the next layer's
+// activation kernel one after the other).
+struct ChainLayout {
+  size_t off_extra, total;
+};
+inline ChainLayout chain_layout(const svdq_params& p, const svdq_params& pn, int64_t M) {
+  ChainLayout L{};
+  const WsLayout W = ws_layout(p, M);
+  L.off_extra = align_up(W.total);
+  const size_t extra = M <= kFewTokens ? (size_t)M * (size_t)p.N * 2
+                                       : (size_t)(p.N / 256) * (size_t)W.Mp * (size_t)pn.rank * 4;
+  L.total = L.off_extra + align_up(extra);
   return L;
 }
 

@@ -87,9 +87,15 @@ struct ActArgs {
   uint8_t* xq;
   uint8_t* xs;
   uint16_t* ux;
-  int ks;   // K split: a cluster of ks CTAs shares one group of 32 tokens
+  int ks;   // K split: ks CTAs share one group of 32 tokens
   int* gemm_cnt;   // GEMM K-split arrival counters to clear (or null)
   int n_cnt;
+  // ks > 8: no cluster; the ks partial down projections of a group meet in
+  // the workspace and the last CTA to arrive adds them (see act_small_ks)
+  int gsplit;
+  unsigned long long epoch;   // nonzero, distinct per call
+  float* upart;               // [groups][ks][32 r] fp32, in mma fragment order
+  unsigned long long* ucnt;   // one arrival word per group
 };
 
 constexpr int kActRows = 32;     // tokens per CTA
@@ -215,44 +221,63 @@ struct QuantDst {
   uint8_t* codes;
   float* sx;
 };
+// max |x| over 16 values (exact: no rounding in a max).
+__device__ __forceinline__ float absmax16(const float (&xh)[16]) {
+  float m8[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fabsf(xh[i]), fabsf(xh[i + 8]));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m8[i] = fmaxf(m8[i], m8[i + 4]);
+  return fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3]));
+}
+
+// NVFP4 block scale code: E4M3_RNE_satfinite(amax / (6 s_gX)), the quotient
+// correctly rounded (r6 = the reciprocal of six_sg when the FMA-corrected
+// route is exact for it, else 0 and an IEEE division).
+__device__ __forceinline__ uint32_t nvfp4_scale_code(float amax, float six_sg, float r6) {
+  const float ratio = r6 != 0.0f ? div_by_recip(amax, six_sg, r6) : __fdiv_rn(amax, six_sg);
+  return cvt_e4m3x2(0.0f, ratio) & 0xFFu;
+}
+
+// The 16 E2M1 codes E2M1_RNE_satfinite(x / d) of one block, packed two per
+// byte (even element in the low nibble): p0 elements 0-7, p1 elements 8-15.
+// d = E4M3(e) s_gX; rd = its round-to-nearest reciprocal when the
+// FMA-corrected quotient is exact, else 0 (IEEE division).  d == 0: all zero.
+__device__ __forceinline__ void nvfp4_codes16(const float (&xh)[16], float d, float rd, uint32_t& p0,
+                                              uint32_t& p1) {
+  p0 = 0; p1 = 0;
+  if (d == 0.0f) return;
+  if (rd != 0.0f) {
+    const uint64_t nd2 = f2_pack(-d, -d), r2 = f2_pack(rd, rd);
+    uint32_t b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float q0, q1;
+      f2_unpack(div2_by_recip(f2_pack(xh[2 * i], xh[2 * i + 1]), nd2, r2), q0, q1);
+      b[i] = cvt_e2m1x2(q1, q0);
+    }
+    p0 = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+    p1 = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      p0 |= cvt_e2m1x2(__fdiv_rn(xh[2 * i + 1], d), __fdiv_rn(xh[2 * i], d)) << (8 * i);
+      p1 |= cvt_e2m1x2(__fdiv_rn(xh[2 * i + 9], d), __fdiv_rn(xh[2 * i + 8], d)) << (8 * i);
+    }
+  }
+}
+
 template <int FMT>
 // dq: NVFP4 per-code tables in shared memory, dq[e] = E4M3(e) * s_gX and
 // dq[256 + e] = its round-to-nearest reciprocal (0 where the FMA-corrected
 // division is not valid); unused for INT4.
 __device__ __forceinline__ void quantize16(const float (&xh)[16], const QuantDst& dst, float six_sg, float r6,
                                            const float* dq) {
-  float m8[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fabsf(xh[i]), fabsf(xh[i + 8]));
-#pragma unroll
-  for (int i = 0; i < 4; ++i) m8[i] = fmaxf(m8[i], m8[i + 4]);
-  float amax = fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3]));
+  float amax = absmax16(xh);
   if constexpr (FMT == SVDQ_NVFP4) {
-    const float ratio = r6 != 0.0f ? div_by_recip(amax, six_sg, r6) : __fdiv_rn(amax, six_sg);
-    const uint32_t e = cvt_e4m3x2(0.0f, ratio) & 0xFFu;
-    const float d = dq[e];
-    const float rd = dq[256 + e];
-    uint32_t p0 = 0, p1 = 0;
-    if (d != 0.0f) {
-      if (rd != 0.0f) {
-        const uint64_t nd2 = f2_pack(-d, -d), r2 = f2_pack(rd, rd);
-        uint32_t b[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float q0, q1;
-          f2_unpack(div2_by_recip(f2_pack(xh[2 * i], xh[2 * i + 1]), nd2, r2), q0, q1);
-          b[i] = cvt_e2m1x2(q1, q0);
-        }
-        p0 = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-        p1 = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          p0 |= cvt_e2m1x2(__fdiv_rn(xh[2 * i + 1], d), __fdiv_rn(xh[2 * i], d)) << (8 * i);
-          p1 |= cvt_e2m1x2(__fdiv_rn(xh[2 * i + 9], d), __fdiv_rn(xh[2 * i + 8], d)) << (8 * i);
-        }
-      }
-    }
+    const uint32_t e = nvfp4_scale_code(amax, six_sg, r6);
+    uint32_t p0, p1;
+    nvfp4_codes16(xh, dq[e], dq[256 + e], p0, p1);
     // activation tile (m / 128, slab): swizzled codes, then the slab's scale atoms
     if (dst.tile) {
       *reinterpret_cast<uint2*>(dst.tile + dst.code_off) = make_uint2(p0, p1);
@@ -310,7 +335,7 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
   if (blockIdx.x == 0 && a.gemm_cnt)
     for (int i = tid; i < a.n_cnt; i += kActThreads) a.gemm_cnt[i] = 0;
   const int KS = a.ks;
-  const int kidx = KS > 1 ? (int)cluster_ctarank() : 0;
+  const int kidx = a.gsplit ? (int)(blockIdx.x % KS) : (KS > 1 ? (int)cluster_ctarank() : 0);
   const int64_t m0 = (int64_t)(blockIdx.x / KS) * kActRows;
   const float s_gx = a.hdr->s_gx;
   const float six_sg = __fmul_rn(6.0f, s_gx);
@@ -469,7 +494,57 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
   for (int t = 0; t < 2; ++t)
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[t][i] += acc2[t][i];
-  if (KS > 1) {
+  if (KS > 1 && a.gsplit) {
+    // partial u of this CTA -> the workspace; count in on the group's arrival
+    // word; the last CTA adds the ks partials in K order (deterministic)
+    const int g = (int)(blockIdx.x / KS);
+    float* mine = a.upart + ((size_t)g * KS + kidx) * (size_t)(32 * r);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int tt = warp + 16 * t;
+      if (tt < n_mma)
+        __stcg(reinterpret_cast<float4*>(mine + (tt * 32 + lane) * 4), make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]));
+    }
+    __threadfence();
+    __syncthreads();
+    __shared__ int last_sh;
+    if (tid == 0) {
+      unsigned long long* w = a.ucnt + g;
+      unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(w), seen;
+      int last = 0;
+      for (;;) {
+        const bool same = (old >> 8) == a.epoch;
+        const unsigned long long cnt = same ? (old & 0xFF) : 0ull;
+        const unsigned long long next = (cnt + 1 == (unsigned long long)KS) ? 0ull : ((a.epoch << 8) | (cnt + 1));
+        seen = atomicCAS(w, old, next);
+        if (seen == old) { last = cnt + 1 == (unsigned long long)KS; break; }
+        old = seen;
+      }
+      last_sh = last;
+    }
+    __syncthreads();
+    if (!last_sh) return;
+    __threadfence();
+    const float* base = a.upart + (size_t)g * KS * (size_t)(32 * r);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int tt = warp + 16 * t;
+      if (tt < n_mma) {
+        const float4* src = reinterpret_cast<const float4*>(base) + tt * 32 + lane;
+        const size_t step = (size_t)(32 * r) / 4;   // float4s per partial
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k0 = 0; k0 < KS; k0 += 8) {         // eight loads in flight, added in order
+          float4 w[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) w[i] = k0 + i < KS ? __ldcg(src + (size_t)(k0 + i) * step) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (k0 + i < KS) { s.x += w[i].x; s.y += w[i].y; s.z += w[i].z; s.w += w[i].w; }
+        }
+        acc[t][0] = s.x; acc[t][1] = s.y; acc[t][2] = s.z; acc[t][3] = s.w;
+      }
+    }
+  } else if (KS > 1) {
     // partial u of this CTA -> its shared memory; CTA 0 adds ranks 1..ks-1 in order
     float* red = reinterpret_cast<float*>(act_smem);
     __syncthreads();   // the last chunk's MMAs have read their operands
@@ -1049,6 +1124,19 @@ constexpr int kEpiWarps = 8;
 constexpr int kP_Threads = 16 * 32;
 constexpr int kEpiChunk = 32 * 128;               // 32 rows x 64 bf16 columns, 128-byte swizzled
 constexpr int kP_Smem = kP_Stages * kS_Size + kEpiWarps * kEpiChunk + 1024;
+// Chained form (the epilogue emits the next layer's quantised input): a
+// 4-deep ring; the tile's X^16 (128 rows x 256 columns bf16, four 64-column
+// swizzled tiles) and this CTA's half of the next layer's L1^T rows for the
+// tile's 256 columns replace the output chunks; the partial down projection
+// (next rank <= 32 columns) sits in TMEM after the scale slots.
+constexpr int kC_Stages = 4;
+constexpr int kC_MaxR = 32;
+constexpr int kC_XHat = 4 * kLRTile;                      // 65536
+constexpr int kC_L1 = 4 * (kC_MaxR / 2) * 128;            // 8192
+constexpr int kC_Smem = kC_Stages * kS_Size + kC_XHat + kC_L1 + 1024;
+constexpr uint32_t kC_UCol = 256 + 48 * kC_Stages;        // 448
+static_assert(kC_UCol + kC_MaxR <= 512, "TMEM columns");
+static_assert((kC_Stages * kS_Size) % 1024 == 0, "X^16 tiles must start on a 1024-byte boundary");
 
 struct PairArgs {
   int64_t M, Mp;
@@ -1065,17 +1153,29 @@ struct PairArgs {
   int ks;                  // K split (few output tiles): items = tiles x ks
   float* part;             // ks > 1: fp32 partial sums [ks][M][N]
   int* cnt;                // ks > 1: arrival counters [tiles][16] (zero between calls)
+  // chained form only: the next layer's input instead of Y
+  const float* nx_inv_lambda;   // next layer's 1/lambda (N values)
+  const BlobHeader* nx_hdr;     // next layer's header (activation tensor scale)
+  uint8_t* nx_atiles;           // next layer's activation tiles [Mp/128][N/256]
+  float* nx_upart;              // partial down projections [N/256][Mp][nx_r]
+  int nx_r;                     // next layer's rank: 0, 16 or 32
 };
 
+template <bool CHAIN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
-    gemm_nvfp4_pair_kernel(const PairArgs g, const __grid_constant__ CUtensorMap tm_y) {
+    gemm_nvfp4_pair_kernel(const PairArgs g, const __grid_constant__ CUtensorMap tm_y,
+                           const __grid_constant__ CUtensorMap tm_l1n) {
+  constexpr int kStages = CHAIN ? kC_Stages : kP_Stages;
   extern __shared__ __align__(1024) uint8_t gsmem_raw[];
-  __shared__ uint64_t landed_bar[kP_Stages], empty_bar[kP_Stages], ready_bar[kP_Stages], accf_bar, acce_bar;
+  __shared__ uint64_t landed_bar[kStages], empty_bar[kStages], ready_bar[kStages], accf_bar, acce_bar;
+  __shared__ uint64_t xready_bar, ufull_bar, l1_bar;   // chained form
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ychunks = smem + kP_Stages * kS_Size;   // one 4 KB output chunk per epilogue warp
+  uint8_t* ychunks = smem + kStages * kS_Size;   // one 4 KB output chunk per epilogue warp
+  uint8_t* xhat = smem + kStages * kS_Size;      // chained form: X^16 tiles, then the L1^T half
+  uint8_t* l1buf = xhat + kC_XHat;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -1091,11 +1191,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
   volatile int* abort_flag = &abort_sh;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kP_Stages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&landed_bar[s], 1); mbar_init(&empty_bar[s], 1); mbar_init(&ready_bar[s], 2 * 4);
     }
     mbar_init(&accf_bar, 1);
     mbar_init(&acce_bar, 2 * kEpiWarps);
+    mbar_init(&xready_bar, 2 * kEpiWarps);
+    mbar_init(&ufull_bar, 1);
+    mbar_init(&l1_bar, 1);
     abort_sh = 0;
     fence_mbar_init();
   }
@@ -1127,8 +1230,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
         const int mt = tile / n_tiles, nt = tile % n_tiles;
         const size_t mb = (size_t)(2 * mt + (int)rank), nb = (size_t)(2 * nt + (int)rank);
         for (int j = 0; j < lr + cpk; ++j, ++it) {
-          const int s = it % kP_Stages;
-          if (!mbar_wait(&empty_bar[s], ((it / kP_Stages) & 1) ^ 1, abort_flag)) { give_up_both(); dead = true; break; }
+          const int s = it % kStages;
+          if (!mbar_wait(&empty_bar[s], ((it / kStages) & 1) ^ 1, abort_flag)) { give_up_both(); dead = true; break; }
           uint8_t* st = smem + s * kS_Size;
           if (j < lr) {
             mbar_arrive_expect_tx(&landed_bar[s], 2 * kLRTile);
@@ -1144,8 +1247,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
         }
       }
       if (*abort_flag) {
-        for (int i = issued - 1; i >= 0 && i >= issued - kP_Stages; --i)
-          mbar_drain(&landed_bar[i % kP_Stages], (i / kP_Stages) & 1);
+        for (int i = issued - 1; i >= 0 && i >= issued - kStages; --i)
+          mbar_drain(&landed_bar[i % kStages], (i / kStages) & 1);
       }
     }
   } else if (warp < 4) {
@@ -1155,13 +1258,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
       const uint32_t id_f4 = idesc_nvf4(256, 256);
       int it = 0, tcount = 0;
       bool dead = false;
+      // chained form: tile t's partial down projection X^16 L1 (M = 256, N =
+      // next rank, K = the tile's 256 columns) once its epilogue has staged
+      // X^16 and the L1^T halves in both CTAs; issued after the next tile's
+      // main loop so the tensor pipe never waits for the epilogue
+      const bool down = CHAIN && g.nx_r > 0;
+      auto down_proj = [&](int t) -> bool {
+        if (!mbar_wait_cluster(&xready_bar, (uint32_t)t & 1u, abort_flag)) { give_up_both(); return false; }
+        tc_fence_after();
+        const uint32_t id_u = idesc_f16_bf16(256, g.nx_r);
+        const uint32_t xa = smem_u32(xhat), la = smem_u32(l1buf);
+        const uint32_t lc = (uint32_t)(g.nx_r / 2) * 128u;   // bytes of one 64-column L1^T chunk
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            mma_f16_pair(tbase + kC_UCol, desc_k_sw128(xa + c * kLRTile + 32 * q), desc_k_sw128(la + c * lc + 32 * q),
+                         id_u, (c | q) != 0);
+        mma_commit_pair(&ufull_bar, 0x3);
+        return true;
+      };
       for (int item = pair; item < num_items && !dead; item += pairs, ++tcount) {
         const int lr = item_lr(item);
         if (!mbar_wait(&acce_bar, (tcount & 1) ^ 1, abort_flag)) { give_up_both(); break; }
         tc_fence_after();
         for (int j = 0; j < lr + cpk; ++j, ++it) {
-          const int s = it % kP_Stages;
-          if (!mbar_wait(&ready_bar[s], (it / kP_Stages) & 1, abort_flag)) { give_up_both(); dead = true; break; }
+          const int s = it % kStages;
+          if (!mbar_wait(&ready_bar[s], (it / kStages) & 1, abort_flag)) { give_up_both(); dead = true; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * kS_Size);
           const uint32_t b_addr = a_addr + kS_B;
@@ -1180,8 +1303,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
           }
           mma_commit_pair(&empty_bar[s], 0x3);
         }
+        if (down && !dead && tcount > 0 && !down_proj(tcount - 1)) dead = true;
         if (!dead) mma_commit_pair(&accf_bar, 0x3);
       }
+      if (down && !dead && tcount > 0) down_proj(tcount - 1);
       if (*abort_flag) {
         mma_commit_pair(&accf_bar, 0x3);
         mbar_drain(&accf_bar, tcount & 1);
@@ -1197,8 +1322,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
     for (int item = pair; item < num_items && !dead; item += pairs) {
       const int lr = item_lr(item);
       for (int j = 0; j < lr + cpk; ++j, ++it) {
-        const int s = it % kP_Stages;
-        if (!mbar_wait(&landed_bar[s], (it / kP_Stages) & 1, abort_flag)) { give_up_both(); dead = true; break; }
+        const int s = it % kStages;
+        if (!mbar_wait(&landed_bar[s], (it / kStages) & 1, abort_flag)) { give_up_both(); dead = true; break; }
         if (j >= lr) {
           const uint8_t* st = smem + s * kS_Size;
           uint32_t wa[16], wb[32];
@@ -1241,6 +1366,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
       float bl[4];   // bias of columns col0 + 32 j + lane
 #pragma unroll
       for (int j = 0; j < 4; ++j) bl[j] = __ldg(g.bias + col0 + 32 * j + lane);
+      if (CHAIN && g.nx_r > 0 && warp == 8 && lane == 0) {
+        // this CTA's half of the next layer's L1^T rows, the tile's 256
+        // columns (the buffer is free: the previous tile's down projection
+        // completed before this warp read its result)
+        const int rh = g.nx_r / 2;
+        mbar_arrive_expect_tx(&l1_bar, (uint32_t)(256 * g.nx_r));
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tma_load_2d(l1buf + c * rh * 128, &tm_l1n, &l1_bar, nt * 256 + 64 * c, (int)rank * rh);
+      }
       if (!mbar_wait(&accf_bar, tcount & 1, abort_flag)) { give_up_both(); break; }
       tc_fence_after();
       uint32_t v[128];
@@ -1253,6 +1388,98 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acce_leader);
       const int64_t row0 = (int64_t)mt * 256 + 128 * rank + q * 32;
+      if constexpr (CHAIN) {
+        // The next layer's input, as its activation kernel would make it from
+        // this layer's bf16 output y: x^ = fp32(y) * inv_lambda', one NVFP4
+        // block per 16 columns (codes and E4M3 scale into the next layer's
+        // activation tile (row tile, K slab nt)), and X^16 = bf16(x^) staged
+        // for the partial down projection.  Rows past M quantise zeros.
+        const int rl = q * 32 + lane;                     // row inside this CTA's 128
+        const bool live = row0 + lane < g.M;
+        const float s_gx = g.nx_hdr->s_gx;
+        const float six_sg = __fmul_rn(6.0f, s_gx);
+        const float r6 = recip_ok(six_sg) ? __frcp_rn(six_sg) : 0.0f;
+        uint8_t* ntile = g.nx_atiles + ((size_t)(2 * mt + (int)rank) * (size_t)n_tiles + (size_t)nt) * kATile;
+        const float4* il4 = reinterpret_cast<const float4*>(g.nx_inv_lambda + col0);
+        uint32_t sc = 0, cw[4];
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {                     // block b: columns 16 b .. 16 b + 15 of this half
+          float xh[16];
+#pragma unroll
+          for (int j4 = 0; j4 < 4; ++j4) {
+            const float4 il = __ldg(il4 + 4 * b + j4);
+            const float ilv[4] = {il.x, il.y, il.z, il.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int e = 16 * b + 4 * j4 + j;
+              const float bb = __shfl_sync(0xffffffffu, bl[e >> 5], e & 31);
+              const float yv = __uint_as_float((uint32_t)bf16_rn(fmaf(alpha, __uint_as_float(v[e]), bb)) << 16);
+              xh[4 * j4 + j] = live ? __fmul_rn(yv, ilv[j]) : 0.0f;
+            }
+          }
+          const uint32_t e8 = nvfp4_scale_code(absmax16(xh), six_sg, r6);
+          const float d = __fmul_rn(e4m3_val(e8), s_gx);
+          const float rd = (d != 0.0f && recip_ok(d)) ? __frcp_rn(d) : 0.0f;
+          nvfp4_codes16(xh, d, rd, cw[2 * (b & 1)], cw[2 * (b & 1) + 1]);
+          sc |= e8 << (8 * (b & 3));
+          if (b & 1)   // two blocks = one 16-byte chunk of the row's codes
+            *reinterpret_cast<uint4*>(ntile + sw128((uint32_t)rl, (uint32_t)(16 * (4 * h + (b >> 1))))) =
+                make_uint4(cw[0], cw[1], cw[2], cw[3]);
+          if ((b & 3) == 3) {   // four scale bytes of one atom
+            *reinterpret_cast<uint32_t*>(ntile + kTileCodes + (2 * h + (b >> 2)) * 512 + (rl & 31) * 16 +
+                                         (rl >> 5) * 4) = sc;
+            sc = 0;
+          }
+          if (g.nx_r > 0) {   // X^16 of the block: two 16-byte pieces of its 64-column tile
+            uint32_t x16[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              x16[i] = (uint32_t)bf16_rn(xh[2 * i]) | ((uint32_t)bf16_rn(xh[2 * i + 1]) << 16);
+            uint8_t* xt = xhat + (2 * h + (b >> 2)) * kLRTile + rl * 128;
+            const int p0 = 2 * (b & 3);
+            *reinterpret_cast<uint4*>(xt + ((p0 ^ (rl & 7)) << 4)) = make_uint4(x16[0], x16[1], x16[2], x16[3]);
+            *reinterpret_cast<uint4*>(xt + (((p0 + 1) ^ (rl & 7)) << 4)) = make_uint4(x16[4], x16[5], x16[6], x16[7]);
+          }
+        }
+        if (g.nx_r > 0) {
+          // hand X^16 (and, from warp 8, the landed L1^T half) to the MMA
+          // thread, then take this tile's partial down projection: lane
+          // quarter q, columns [h r/2, (h + 1) r/2) of the next rank
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (warp == 8 && !mbar_wait(&l1_bar, tcount & 1, abort_flag)) give_up_both();
+            mbar_arrive_cluster_release(mapa_shared(smem_u32(&xready_bar), 0));
+          }
+          __syncwarp();
+          if (!mbar_wait(&ufull_bar, tcount & 1, abort_flag)) { give_up_both(); break; }
+          tc_fence_after();
+          const int rh = g.nx_r / 2;
+          const uint32_t ua = tbase + ((uint32_t)(q * 32) << 16) + kC_UCol + (uint32_t)(h * rh);
+          float* dst = g.nx_upart + ((size_t)nt * (size_t)g.Mp + (size_t)(row0 + lane)) * g.nx_r + h * rh;
+          if (rh == 16) {
+            uint32_t uv[16];
+            tmem_ld_16cols(ua, uv);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              reinterpret_cast<float4*>(dst)[c] =
+                  make_float4(__uint_as_float(uv[4 * c]), __uint_as_float(uv[4 * c + 1]),
+                              __uint_as_float(uv[4 * c + 2]), __uint_as_float(uv[4 * c + 3]));
+          } else {
+            uint32_t uv[8];
+            tmem_ld_8cols(ua, uv);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              reinterpret_cast<float4*>(dst)[c] =
+                  make_float4(__uint_as_float(uv[4 * c]), __uint_as_float(uv[4 * c + 1]),
+                              __uint_as_float(uv[4 * c + 2]), __uint_as_float(uv[4 * c + 3]));
+          }
+          tc_fence_before();
+        }
+        continue;
+      }
       if (g.ks > 1) {
         // K split: this item's raw sums -> part[kq]; the warp that completes a
         // region adds the ks partials in K order (deterministic), then applies
@@ -1354,16 +1581,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
   }
 }
 
+// ------------------------------------------------------------ chained form: next low-rank input
+// u'[m, i] = (sum over the output tile columns t, in order, of the chained
+// GEMM's partial X^16 L1 [t][m][i]) / (s_gX s_gW) of the next layer, written
+// as bf16 hi + lo into the next layer's low-rank input tiles in the format
+// its activation kernel writes ([u'_hi | u'_lo | 0 pad], 128 x 64 swizzled
+// tiles).  One thread per (token, 4 columns of the low-rank row).
+constexpr int kCU_Threads = 256;
+__global__ void __launch_bounds__(kCU_Threads) chain_u_kernel(const float* upart, int tiles, int64_t Mp, int r,
+                                                              int lrw, const BlobHeader* nx_hdr, uint8_t* ux) {
+  griddep_wait();   // the partials come from the chained GEMM
+  const int per_row = lrw / 4;
+  const int64_t idx = (int64_t)blockIdx.x * kCU_Threads + threadIdx.x;
+  if (idx >= Mp * per_row) return;
+  const int64_t m = idx / per_row;
+  const int j = (int)(idx % per_row);
+  const int c4 = r / 4;
+  if (j >= c4 && j < 2 * c4) return;   // the lo half is written with its hi half
+  uint8_t* const utile = ux + (size_t)(m / 128) * (size_t)(lrw / 64) * kLRTile;
+  auto store4 = [&](int col, uint32_t w0, uint32_t w1) {   // 4 bf16 at columns col .. col + 3
+    uint8_t* tile = utile + (size_t)(col / 64) * kLRTile;
+    *reinterpret_cast<uint2*>(tile + sw128((uint32_t)(m % 128), (uint32_t)(col % 64) * 2)) = make_uint2(w0, w1);
+  };
+  if (j >= 2 * c4) {
+    store4(4 * j, 0u, 0u);
+    return;
+  }
+  const float4* src = reinterpret_cast<const float4*>(upart + (size_t)m * r) + j;
+  const size_t tstride = (size_t)Mp * (size_t)r / 4;   // float4s per tile column
+  float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  int t = 0;
+  for (; t + 8 <= tiles; t += 8) {   // eight loads in flight, added in order
+    float4 w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = __ldcg(src + (size_t)(t + i) * tstride);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { acc.x += w[i].x; acc.y += w[i].y; acc.z += w[i].z; acc.w += w[i].w; }
+  }
+  for (; t < tiles; ++t) {
+    const float4 w = __ldcg(src + (size_t)t * tstride);
+    acc.x += w.x; acc.y += w.y; acc.z += w.z; acc.w += w.w;
+  }
+  const float inv_alpha = 1.0f / (nx_hdr->s_gx * nx_hdr->s_gw);
+  const float v[4] = {acc.x * inv_alpha, acc.y * inv_alpha, acc.z * inv_alpha, acc.w * inv_alpha};
+  uint32_t hi[2], lo[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const uint32_t h0 = bf16_rn(v[2 * k]), h1 = bf16_rn(v[2 * k + 1]);
+    const uint32_t l0 = bf16_rn(v[2 * k] - __uint_as_float(h0 << 16));
+    const uint32_t l1 = bf16_rn(v[2 * k + 1] - __uint_as_float(h1 << 16));
+    hi[k] = h0 | (h1 << 16);
+    lo[k] = l0 | (l1 << 16);
+  }
+  store4(4 * j, hi[0], hi[1]);
+  store4(r + 4 * j, lo[0], lo[1]);
+}
+
 // ------------------------------------------------------------ kernel 2, NVFP4, few tokens
-// Up to 16 tokens: the layer streams its weights, so the weight tile is the
+// Up to 128 tokens: the layer streams its weights, so the weight tile is the
 // 128-row A operand of a 1-CTA kind::mxf4nvf4 MMA and the tokens are a
-// 16-column B operand (M = 128 output features, N = 16 tokens, K = 64):
-// D[feature, token] accumulates in 16 TMEM columns.  One CTA per (128-feature
+// TOK-column B operand (M = 128 output features, N = TOK = 16, 64 or 128
+// tokens, K = 64): D[feature, token] accumulates in TOK TMEM columns.  One CTA per (128-feature
 // tile, K part); with ks > 1 K parts add through fp32 partials (the last CTA
 // of a tile adds them in K order, as in the pair kernel).
 // Per 256-wide K slab a ring stage holds the tile's codes (16 KB) and its
-// 128 rows of scale atoms (2 KB), and the first 16 rows of the activation
-// tile's codes (2 KB) and its scale atoms (2 KB): four bulk copies.  The
+// 128 rows of scale atoms (2 KB), and the first TOK rows of the activation
+// tile's codes (TOK x 128 bytes) and its scale atoms (2 KB): four bulk copies.  The
 // weight halves of the first stages are issued before the wait for the
 // activation kernel.  Four scale warps (one per TMEM lane quarter) move a
 // landed stage's eight scale atoms to its TMEM slot with tcgen05.st and
@@ -1371,22 +1654,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
 // (with the scale copies on the MMA thread, the measured issue cost was
 // ~0.5 us per stage, slower than the weight stream).  The low-rank up
 // projection u' L2 runs last as kind::f16 K-steps (A = the L2 tile of the 128
-// features, B = the first 16 rows of the low-rank input tile) into the same
+// features, B = the first TOK rows of the low-rank input tile) into the same
 // accumulator.
 // Warps: 0 producer, 1 TMEM owner + MMA issuer, 2-5 scale warps, then the
 // epilogue (lane quarters).
-constexpr int kSM_Tokens = 16;
-constexpr int kSM_Stage = kTileCodes + 2048 + kSM_Tokens * 128 + 2048;   // 22528
-constexpr int kSM_Stages = 9;
+constexpr int kSM_MaxTokens = (int)kFewTokens;
 constexpr int kSM_Threads = 6 * 32;
-constexpr int kSM_Smem = kSM_Stages * kSM_Stage + 1024;
-// stage offsets: [W codes | W scales | X codes (16 rows) | X scales]
-constexpr int kSM_WS = kTileCodes, kSM_X = kTileCodes + 2048, kSM_XS = kSM_X + kSM_Tokens * 128;
+// stage: [W codes | W scales | X codes (TOK rows) | X scales]
+SVDQ_HD constexpr int sm_stage(int tok) { return kTileCodes + 2048 + tok * 128 + 2048; }
+SVDQ_HD constexpr int sm_stages(int tok) { return (232448 - 4096 - 1024) / sm_stage(tok) > 9 ? 9 : (232448 - 4096 - 1024) / sm_stage(tok); }
+SVDQ_HD constexpr int sm_smem(int tok) { return sm_stages(tok) * sm_stage(tok) + 1024; }
+constexpr int kSM_MaxStages = 9;
 
+template <int TOK>
 __global__ void __launch_bounds__(kSM_Threads, 1)
     gemm_nvfp4_small_kernel(const PairArgs g) {
+  constexpr int kSM_Tokens = TOK;
+  constexpr int kSM_Stage = sm_stage(TOK);
+  constexpr int kSM_Stages = sm_stages(TOK);
+  constexpr int kSM_WS = kTileCodes, kSM_X = kTileCodes + 2048, kSM_XS = kSM_X + TOK * 128;
+  constexpr uint32_t kSF0 = TOK < 32 ? 32u : (uint32_t)TOK;   // scale slots after the accumulator's columns
   extern __shared__ __align__(1024) uint8_t gsmem_raw[];
-  __shared__ uint64_t full_bar[kSM_Stages], empty_bar[kSM_Stages], ready_bar[kSM_Stages], accf_bar;
+  __shared__ uint64_t full_bar[kSM_MaxStages], empty_bar[kSM_MaxStages], ready_bar[kSM_MaxStages], accf_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -1474,7 +1763,7 @@ __global__ void __launch_bounds__(kSM_Threads, 1)
         const uint32_t a_addr = smem_u32(smem + s * kSM_Stage);
         const uint32_t b_addr = a_addr + kSM_X;
         if (j < cpk) {
-          const uint32_t sfa_t = tbase + 32 + 32 * s, sfb_t = sfa_t + 16;   // the stage's scale slot
+          const uint32_t sfa_t = tbase + kSF0 + 32 * s, sfb_t = sfa_t + 16;   // the stage's scale slot
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             mma_nvf4(tbase, desc_k_sw128(a_addr + 32 * q), desc_k_sw128(b_addr + 32 * q), id_f4, sfa_t + 4 * q,
@@ -1506,13 +1795,13 @@ __global__ void __launch_bounds__(kSM_Threads, 1)
             w[4 * k] = a4.x; w[4 * k + 1] = a4.y; w[4 * k + 2] = a4.z; w[4 * k + 3] = a4.w;
           }
           tc_fence_after();
-          tmem_st_16cols(lane_base + 32 + 32 * s, w);
+          tmem_st_16cols(lane_base + kSF0 + 32 * s, w);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint4 b4 = *reinterpret_cast<const uint4*>(st + kSM_XS + 512 * k + lane * 16);
             w[4 * k] = b4.x; w[4 * k + 1] = b4.y; w[4 * k + 2] = b4.z; w[4 * k + 3] = b4.w;
           }
-          tmem_st_16cols(lane_base + 32 + 32 * s + 16, w);
+          tmem_st_16cols(lane_base + kSF0 + 32 * s + 16, w);
           tmem_st_wait();
           tc_fence_before();
         }
@@ -1526,35 +1815,46 @@ __global__ void __launch_bounds__(kSM_Threads, 1)
     const float b = __ldg(g.bias + n);
     if (__all_sync(0xffffffffu, mbar_wait(&accf_bar, 0, abort_flag))) {
       tc_fence_after();
-      uint32_t v[16];
-      asm volatile(
-          "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-          "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-            "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-          : "r"(tbase + ((uint32_t)(q * 32) << 16)));
-      tmem_ld_wait();
       const int M = (int)g.M;
-      if (ks == 1) {
+      int* cnt = g.cnt + (size_t)nt * 4 + q;
+      for (int m0 = 0; m0 < TOK && m0 < M; m0 += 16) {
+        uint32_t v[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+            : "r"(tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)m0));
+        tmem_ld_wait();
 #pragma unroll
-        for (int m = 0; m < kSM_Tokens; ++m)
-          if (m < M) g.Y[(size_t)m * g.N + n] = bf16_rn(fmaf(alpha, __uint_as_float(v[m]), b));
-      } else {
-        // raw sums -> part[kq]; the warp completing its 32 features adds the parts in K order
-#pragma unroll
-        for (int m = 0; m < kSM_Tokens; ++m)
-          if (m < M) __stcg(g.part + ((size_t)kq * g.M + m) * g.N + n, __uint_as_float(v[m]));
+        for (int j = 0; j < 16; ++j) {
+          const int m = m0 + j;
+          if (m < M) {
+            if (ks == 1) g.Y[(size_t)m * g.N + n] = bf16_rn(fmaf(alpha, __uint_as_float(v[j]), b));
+            else __stcg(g.part + ((size_t)kq * g.M + m) * g.N + n, __uint_as_float(v[j]));
+          }
+        }
+      }
+      if (ks > 1) {
+        // the warp completing its 32 features adds the K parts in order
         __threadfence();
         __syncwarp();
-        int* cnt = g.cnt + (size_t)nt * 4 + q;
         int old = 0;
         if (lane == 0) old = atomicAdd(cnt, 1);
         old = __shfl_sync(0xffffffffu, old, 0);
         if (old == ks - 1) {
           __threadfence();
+          // eight tokens' ks loads in flight at once, each token's added in K order
+#pragma unroll 8
           for (int m = 0; m < M; ++m) {
+            float pk[kMaxKSplit];
+#pragma unroll
+            for (int k = 0; k < kMaxKSplit; ++k)
+              pk[k] = k < ks ? __ldcg(g.part + ((size_t)k * g.M + m) * g.N + n) : 0.0f;
             float t = 0.0f;
-            for (int k = 0; k < ks; ++k) t += __ldcg(g.part + ((size_t)k * g.M + m) * g.N + n);
+#pragma unroll
+            for (int k = 0; k < kMaxKSplit; ++k)
+              if (k < ks) t += pk[k];
             g.Y[(size_t)m * g.N + n] = bf16_rn(fmaf(alpha, t, b));
           }
           if (lane == 0) *cnt = 0;   // ready for the next call
@@ -2060,10 +2360,16 @@ svdq_status device_ready() {
     d.sms = prop.multiProcessorCount;
     if (d.ok) {
       const int i4_smem = dev::kI4Smem;
-      d.ok = cudaFuncSetAttribute(dev::gemm_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      d.ok = cudaFuncSetAttribute(dev::gemm_nvfp4_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   dev::kP_Smem) == cudaSuccess &&
-             cudaFuncSetAttribute(dev::gemm_nvfp4_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  dev::kSM_Smem) == cudaSuccess &&
+             cudaFuncSetAttribute(dev::gemm_nvfp4_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  dev::kC_Smem) == cudaSuccess &&
+             cudaFuncSetAttribute(dev::gemm_nvfp4_small_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  dev::sm_smem(16)) == cudaSuccess &&
+             cudaFuncSetAttribute(dev::gemm_nvfp4_small_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  dev::sm_smem(64)) == cudaSuccess &&
+             cudaFuncSetAttribute(dev::gemm_nvfp4_small_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  dev::sm_smem(128)) == cudaSuccess &&
              cudaFuncSetAttribute(dev::gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   i4_smem) == cudaSuccess;
       const int act_smem = dev::kActSmemMax;
@@ -2123,11 +2429,24 @@ std::atomic<unsigned long long> g_act_epoch{
 template <int FMT>
 cudaError_t launch_act(const svdq_params* p, dev::ActArgs a, int64_t Mp, cudaStream_t stream) {
   a.ks = act_k_split(Mp, p->K);
+  a.gsplit = 0;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(Mp / dev::kActRows * a.ks));
   cfg.blockDim = dim3(dev::kActThreads);
-  cfg.dynamicSmemBytes = (size_t)dev::act_smem_bytes(p->rank, p->K / a.ks);
   cfg.stream = stream;
+  if (FMT == SVDQ_NVFP4 && a.upart != nullptr) {
+    // few live 32-token groups: only they run (rows past them are never read
+    // for live tokens), ks > 8 CTAs each, partials through the workspace
+    a.ks = act_small_ks(a.M, p->K);
+    a.gsplit = 1;
+    a.epoch = g_act_epoch.fetch_add(1) & 0x00FFFFFFFFFFFFFFull;
+    if (a.epoch == 0) a.epoch = g_act_epoch.fetch_add(1) & 0x00FFFFFFFFFFFFFFull;
+    cfg.gridDim = dim3((unsigned)((a.M + dev::kActRows - 1) / dev::kActRows * a.ks));
+    cfg.dynamicSmemBytes = (size_t)dev::act_smem_bytes(p->rank, p->K / a.ks);
+    if (p->act_dtype == SVDQ_BF16) return cudaLaunchKernelEx(&cfg, dev::act_quant_kernel<FMT, SVDQ_BF16>, a);
+    return cudaLaunchKernelEx(&cfg, dev::act_quant_kernel<FMT, SVDQ_F16>, a);
+  }
+  cfg.gridDim = dim3((unsigned)(Mp / dev::kActRows * a.ks));
+  cfg.dynamicSmemBytes = (size_t)dev::act_smem_bytes(p->rank, p->K / a.ks);
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = (unsigned)a.ks;
@@ -2171,6 +2490,12 @@ svdq_status launch_quantize(const svdq_params* p, const void* blob_dev, const vo
   a.ux = reinterpret_cast<uint16_t*>(ws + W.off_ux);
   a.gemm_cnt = W.off_cnt > W.off_part ? reinterpret_cast<int*>(ws + W.off_cnt) : nullptr;
   a.n_cnt = (p->N / 256) * (int)(W.Mp / 256) * 16;
+  // the 32-token kernel's workspace K split (NVFP4, few tokens; see ws_layout)
+  const bool gsplit = p->fmt == SVDQ_NVFP4 && M <= 256 && W.off_ucnt > W.off_upart;
+  a.upart = gsplit ? reinterpret_cast<float*>(ws + W.off_upart) : nullptr;
+  a.ucnt = gsplit ? reinterpret_cast<unsigned long long*>(ws + W.off_ucnt) : nullptr;
+  a.gsplit = 0;
+  a.epoch = 0;
   // NVFP4 above 256 tokens: the 128-token-tile kernel (tcgen05 down projection).
   // Up to 256 tokens the 32-token kernel wins: its latency chain per call is
   // shorter (measured 12-22 us against 20-25 us at one token on the VAR shapes).
@@ -2226,7 +2551,7 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
   const int K = p->K, N = p->N, r = p->rank, lrw = lr_width(*p);
   const bool fp4 = p->fmt == SVDQ_NVFP4;
   if (fp4) {
-    dev::PairArgs g;
+    dev::PairArgs g{};
     g.M = M; g.Mp = W.Mp; g.N = N; g.K = K;
     g.lr_iters = r > 0 ? lrw / 64 : 0;
     g.k_iters = K / 256;
@@ -2242,9 +2567,9 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
       return cuda_fail(cudaErrorInvalidValue, "tensor map encode (Y)");
     g.part = reinterpret_cast<float*>(ws + W.off_part);
     g.cnt = reinterpret_cast<int*>(ws + W.off_cnt);
-    if (M <= dev::kSM_Tokens) {
-      // few tokens: the weight tile as the A operand of a 1-CTA MMA, K split
-      // over idle SMs when the workspace holds the partials
+    if (M <= dev::kSM_MaxTokens) {
+      // up to 128 tokens: the weight tile as the A operand of a 1-CTA MMA, K
+      // split over idle SMs when the workspace holds the partials
       const int n_tiles = N / 128;
       g.ks = 1;
       if (W.off_cnt > W.off_part)
@@ -2254,14 +2579,23 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3((unsigned)(n_tiles * g.ks));
       cfg.blockDim = dim3(dev::kSM_Threads);
-      cfg.dynamicSmemBytes = dev::kSM_Smem;
       cfg.stream = stream;
       cudaLaunchAttribute at[1];
       at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
       at[0].val.programmaticStreamSerializationAllowed = 1;
       cfg.attrs = at;
       cfg.numAttrs = 1;
-      const cudaError_t e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_small_kernel, g);
+      cudaError_t e;
+      if (M <= 16) {
+        cfg.dynamicSmemBytes = dev::sm_smem(16);
+        e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_small_kernel<16>, g);
+      } else if (M <= 64) {
+        cfg.dynamicSmemBytes = dev::sm_smem(64);
+        e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_small_kernel<64>, g);
+      } else {
+        cfg.dynamicSmemBytes = dev::sm_smem(128);
+        e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_small_kernel<128>, g);
+      }
       if (e != cudaSuccess) return cuda_fail(e, "gemm_nvfp4_small_kernel launch");
       return launch_status("gemm_nvfp4_small_kernel launch");
     }
@@ -2283,7 +2617,7 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_pair_kernel, g, tm_y);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_pair_kernel<false>, g, tm_y, tm_y);
     if (e != cudaSuccess) return cuda_fail(e, "gemm_nvfp4_pair_kernel launch");
     return launch_status("gemm_nvfp4_pair_kernel launch");
   }
@@ -2329,6 +2663,75 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
   return launch_status("gemm kernel launch");
 }
 
+// This layer's GEMM writing the next layer's quantised input into ws_next
+// (its activation tiles and low-rank input tiles) instead of Y.
+svdq_status launch_gemm_chain(const svdq_params* p, const void* blob_dev, int64_t M, const svdq_params* pn,
+                              const void* blob_next, void* workspace, void* ws_next, cudaStream_t stream) {
+  const ChainLayout C = chain_layout(*p, *pn, M);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (M <= kFewTokens) {
+    // a few tokens: Y is at most 128 rows, so it goes through the workspace
+    // to the next layer's activation kernel
+    void* y = ws + C.off_extra;
+    const svdq_status st = launch_gemm(p, blob_dev, M, y, workspace, stream);
+    if (st != SVDQ_OK) return st;
+    return launch_quantize(pn, blob_next, y, M, ws_next, stream);
+  }
+  const WsLayout W = ws_layout(*p, M);
+  const WsLayout Wn = ws_layout(*pn, M);
+  const BlobLayout B = blob_layout(*p);
+  const BlobLayout Bn = blob_layout(*pn);
+  const uint8_t* blob = static_cast<const uint8_t*>(blob_dev);
+  const uint8_t* nblob = static_cast<const uint8_t*>(blob_next);
+  uint8_t* wsn = static_cast<uint8_t*>(ws_next);
+  const int K = p->K, N = p->N, r = p->rank, lrw = lr_width(*p), rn = pn->rank;
+  dev::PairArgs g{};
+  g.M = M; g.Mp = W.Mp; g.N = N; g.K = K;
+  g.lr_iters = r > 0 ? lrw / 64 : 0;
+  g.k_iters = K / 256;
+  g.atiles = ws + W.off_xq;
+  g.wtiles = blob + B.off_wq;
+  g.utiles = ws + W.off_ux;
+  g.l2tiles = blob + B.off_l2x;
+  g.bias = reinterpret_cast<const float*>(blob + B.off_bias);
+  g.hdr = reinterpret_cast<const BlobHeader*>(blob);
+  g.ks = 1;
+  g.nx_inv_lambda = reinterpret_cast<const float*>(nblob + Bn.off_inv_lambda);
+  g.nx_hdr = reinterpret_cast<const BlobHeader*>(nblob);
+  g.nx_atiles = wsn + Wn.off_xq;
+  g.nx_upart = reinterpret_cast<float*>(ws + C.off_extra);
+  g.nx_r = rn;
+  CUtensorMap tm_l1n{};
+  if (rn > 0 && !make_map(&tm_l1n, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, nblob + Bn.off_l1t, (uint64_t)N, (uint64_t)rn,
+                          (uint64_t)N * 2, 64, (uint32_t)(rn / 2)))
+    return cuda_fail(cudaErrorInvalidValue, "tensor map encode (next layer L1)");
+  const int tiles = (N / 256) * (int)(W.Mp / 256);
+  const int pairs = std::max(1, std::min(tiles, num_sms() / 2));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(dev::kP_Threads);
+  cfg.dynamicSmemBytes = dev::kC_Smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_pair_kernel<true>, g, tm_l1n, tm_l1n);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm_nvfp4_pair_kernel (chained) launch");
+  if (rn > 0) {
+    const int lrw_n = lr_width(*pn);
+    const int64_t items = Wn.Mp * (lrw_n / 4);
+    cfg.gridDim = dim3((unsigned)((items + dev::kCU_Threads - 1) / dev::kCU_Threads));
+    cfg.blockDim = dim3(dev::kCU_Threads);
+    cfg.dynamicSmemBytes = 0;
+    e = cudaLaunchKernelEx(&cfg, dev::chain_u_kernel, (const float*)g.nx_upart, N / 256, (int64_t)Wn.Mp, rn, lrw_n,
+                           g.nx_hdr, wsn + Wn.off_ux);
+    if (e != cudaSuccess) return cuda_fail(e, "chain_u_kernel launch");
+  }
+  return launch_status("chained gemm launch");
+}
+
 }  // namespace
 
 extern "C" {
@@ -2349,6 +2752,22 @@ svdq_status svdq_gemm(const svdq_params* p, const void* blob_dev, int64_t M, voi
   if (!Y) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(Y)) return SVDQ_ERR_ALIGNMENT;
   return launch_gemm(p, blob_dev, M, Y, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+svdq_status svdq_gemm_chain(const svdq_params* p, const void* blob_dev, int64_t M, const svdq_params* p_next,
+                            const void* blob_next_dev, void* workspace, size_t ws_bytes, void* ws_next,
+                            size_t ws_next_bytes, svdq_stream stream) {
+  svdq_status st = check_params_dev(p_next);
+  if (st != SVDQ_OK) return st;
+  if ((st = chain_supported(*p, *p_next)) != SVDQ_OK) return st;
+  st = common_checks(p, blob_dev, M, workspace, ws_bytes);
+  if (st != SVDQ_OK || M == 0) return st;
+  if (ws_bytes < chain_layout(*p, *p_next, M).total) return SVDQ_ERR_WORKSPACE;
+  if (!blob_next_dev || !ws_next) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(blob_next_dev) || !aligned16(ws_next)) return SVDQ_ERR_ALIGNMENT;
+  if (ws_next_bytes < ws_layout(*p_next, M).total) return SVDQ_ERR_WORKSPACE;
+  return launch_gemm_chain(p, blob_dev, M, p_next, blob_next_dev, workspace, ws_next,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 svdq_status svdq_linear(const svdq_params* p, const void* blob_dev, const void* X, int64_t M, void* Y,

@@ -418,6 +418,12 @@ size_t svdq_workspace_bytes(const svdq_params* p, int64_t M) {
   return ws_layout(*p, M).total;
 }
 
+size_t svdq_chain_workspace_bytes(const svdq_params* p, const svdq_params* p_next, int64_t M) {
+  if (check_params(p) != SVDQ_OK || check_params(p_next) != SVDQ_OK || M < 0) return 0;
+  if (chain_supported(*p, *p_next) != SVDQ_OK) return 0;
+  return chain_layout(*p, *p_next, M).total;
+}
+
 const char* svdq_status_string(svdq_status s) {
   switch (s) {
     case SVDQ_OK: return "ok";

@@ -137,11 +137,13 @@ def test_status_word_clean(gpu):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp16"])
-@pytest.mark.parametrize("M", [1, 5, 64])
+@pytest.mark.parametrize("M", [1, 5, 16, 17, 64, 65, 100, 128])
 def test_small_m_split_k(gpu, dtype, M):
-    """Few tokens and few output tiles: the NVFP4 GEMM splits K over several
-    CTA pairs and adds the partial sums in K order.  Two calls in a row give
-    identical bits (the arrival counters reset) and match the oracle."""
+    """Few tokens: the NVFP4 GEMM with the weight tile as the A operand and
+    16, 64 or 128 token columns (each width at its edges), splitting K over
+    idle SMs up to 64 tokens and adding the partial sums in K order.  Two
+    calls in a row give identical bits (the arrival counters reset) and match
+    the oracle."""
     wl = synth.custom_workload(M, 2048, 1024, 32, "nvfp4", dtype, n_out=6, factor=60.0, seed=40 + M)
     pp = G.prepare(wl)
     a = G.run_gpu(pp, wl.X)
@@ -152,10 +154,12 @@ def test_small_m_split_k(gpu, dtype, M):
 
 @pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
-def test_max_rank(gpu, fmt, dtype):
+@pytest.mark.parametrize("M", [100, 200])
+def test_max_rank(gpu, fmt, dtype, M):
     """Rank 128 (the largest allowed): several low-rank K-steps (up to 6 for
-    fp16's three segments) and the activation kernel's two-buffer L1 ring."""
-    wl = synth.custom_workload(200, 1024, 512, 128, fmt, dtype, n_out=8, factor=40.0, seed=77)
+    fp16's three segments) and the activation kernel's two-buffer L1 ring,
+    through both NVFP4 GEMM kernels (up to 128 tokens and above)."""
+    wl = synth.custom_workload(M, 1024, 512, 128, fmt, dtype, n_out=8, factor=40.0, seed=77 + M)
     pp = G.prepare(wl)
     run = G.run_gpu(pp, wl.X)
     G.compare(pp, wl.X, run)

@@ -139,16 +139,17 @@ SVDQ_HD inline int act_nv_ks(int64_t Mp, int K) {
 }
 
 // NVFP4 up to 256 tokens (the 32-token activation kernel): with few live
-// 32-token groups, ks CTAs split a group's K range (a power of two dividing
-// K / 256, at most kActGMaxKs).  Up to 8 they form a cluster and add their
-// partial down projections through distributed shared memory; above 8 the
-// partials meet in the workspace ([groups][ks][32][r] fp32 plus one 64-bit
+// 32-token groups and K >= 8192, ks CTAs split a group's K range (a power of
+// two dividing K / 256, at most kActGMaxKs).  Clusters of up to 8 add their partial down
+// projections through distributed shared memory; above 8 the ks / 8 cluster
+// sums meet in the workspace ([groups][ks / 8][32][r] fp32 plus one 64-bit
 // arrival word per group, tagged per call like the 128-token kernel's).
 constexpr int kActGMaxKs = 32;
 constexpr int kActClusterKs = 8;
 SVDQ_HD inline int act_small_ks(int64_t M, int K) {
   const int64_t groups = (M + 31) / 32;
   const int chunks = K / 256;
+  if (chunks < 4 * kActClusterKs) return 1;   // a cluster of 8 leaves <= 3 slabs per CTA: no workspace split
   int ks = 1;
   while (ks < kActGMaxKs && groups * ks * 2 <= kActSizingSMs && chunks % (ks * 2) == 0) ks *= 2;
   return ks;
@@ -186,7 +187,7 @@ inline WsLayout ws_layout(const svdq_params& p, int64_t M) {
     const int ks = act_small_ks(M, p.K);
     if (ks > kActClusterKs && p.rank > 0) {
       const size_t groups = (size_t)((M + 31) / 32);
-      off = align_up(off + groups * (size_t)ks * 32 * (size_t)p.rank * 4);
+      off = align_up(off + groups * (size_t)(ks / kActClusterKs) * 32 * (size_t)p.rank * 4);
       L.off_ucnt = off;
       off = align_up(off + groups * 8);
     }

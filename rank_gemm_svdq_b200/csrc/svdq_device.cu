@@ -90,11 +90,12 @@ struct ActArgs {
   int ks;   // K split: ks CTAs share one group of 32 tokens
   int* gemm_cnt;   // GEMM K-split arrival counters to clear (or null)
   int n_cnt;
-  // ks > 8: no cluster; the ks partial down projections of a group meet in
-  // the workspace and the last CTA to arrive adds them (see act_small_ks)
-  int gsplit;
+  // workspace split (the GS kernels, ks > 8): clusters of 8 add their partial
+  // down projections through distributed shared memory, and the ks / 8
+  // cluster sums of a group meet in the workspace, where the last to arrive
+  // adds them (see act_small_ks)
   unsigned long long epoch;   // nonzero, distinct per call
-  float* upart;               // [groups][ks][32 r] fp32, in mma fragment order
+  float* upart;               // [groups][ks / 8][32 r] fp32, in mma fragment order
   unsigned long long* ucnt;   // one arrival word per group
 };
 
@@ -221,6 +222,8 @@ struct QuantDst {
   uint8_t* codes;
   float* sx;
 };
+// The steps of quantize16's NVFP4 branch as separate helpers, for the chained
+// GEMM epilogue (the activation kernel keeps its own inline copy).
 // max |x| over 16 values (exact: no rounding in a max).
 __device__ __forceinline__ float absmax16(const float (&xh)[16]) {
   float m8[8];
@@ -273,11 +276,38 @@ template <int FMT>
 // division is not valid); unused for INT4.
 __device__ __forceinline__ void quantize16(const float (&xh)[16], const QuantDst& dst, float six_sg, float r6,
                                            const float* dq) {
-  float amax = absmax16(xh);
+  float m8[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fabsf(xh[i]), fabsf(xh[i + 8]));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m8[i] = fmaxf(m8[i], m8[i + 4]);
+  float amax = fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3]));
   if constexpr (FMT == SVDQ_NVFP4) {
-    const uint32_t e = nvfp4_scale_code(amax, six_sg, r6);
-    uint32_t p0, p1;
-    nvfp4_codes16(xh, dq[e], dq[256 + e], p0, p1);
+    const float ratio = r6 != 0.0f ? div_by_recip(amax, six_sg, r6) : __fdiv_rn(amax, six_sg);
+    const uint32_t e = cvt_e4m3x2(0.0f, ratio) & 0xFFu;
+    const float d = dq[e];
+    const float rd = dq[256 + e];
+    uint32_t p0 = 0, p1 = 0;
+    if (d != 0.0f) {
+      if (rd != 0.0f) {
+        const uint64_t nd2 = f2_pack(-d, -d), r2 = f2_pack(rd, rd);
+        uint32_t b[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float q0, q1;
+          f2_unpack(div2_by_recip(f2_pack(xh[2 * i], xh[2 * i + 1]), nd2, r2), q0, q1);
+          b[i] = cvt_e2m1x2(q1, q0);
+        }
+        p0 = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+        p1 = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          p0 |= cvt_e2m1x2(__fdiv_rn(xh[2 * i + 1], d), __fdiv_rn(xh[2 * i], d)) << (8 * i);
+          p1 |= cvt_e2m1x2(__fdiv_rn(xh[2 * i + 9], d), __fdiv_rn(xh[2 * i + 8], d)) << (8 * i);
+        }
+      }
+    }
     // activation tile (m / 128, slab): swizzled codes, then the slab's scale atoms
     if (dst.tile) {
       *reinterpret_cast<uint2*>(dst.tile + dst.code_off) = make_uint2(p0, p1);
@@ -320,7 +350,7 @@ __device__ __forceinline__ void quantize16(const float (&xh)[16], const QuantDst
 // double-buffered, so a chunk costs one __syncthreads.  The down projection
 // u = X^16 L1 runs on mma.sync (m16n8k16, fp32 accumulate): 2 x r/8 tiles of
 // 16 tokens x 8 ranks, tile t on warp t % 16.
-template <int FMT, int DT>
+template <int FMT, int DT, bool GS>
 __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs a) {
   extern __shared__ __align__(16) uint16_t act_smem[];
   const int K = a.K, r = a.r;
@@ -335,7 +365,9 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
   if (blockIdx.x == 0 && a.gemm_cnt)
     for (int i = tid; i < a.n_cnt; i += kActThreads) a.gemm_cnt[i] = 0;
   const int KS = a.ks;
-  const int kidx = a.gsplit ? (int)(blockIdx.x % KS) : (KS > 1 ? (int)cluster_ctarank() : 0);
+  // K part of this CTA; with the workspace split the ks parts run as ks / 8
+  // clusters of 8 (cluster rank = kidx % 8)
+  const int kidx = GS ? (int)(blockIdx.x % KS) : (KS > 1 ? (int)cluster_ctarank() : 0);
   const int64_t m0 = (int64_t)(blockIdx.x / KS) * kActRows;
   const float s_gx = a.hdr->s_gx;
   const float six_sg = __fmul_rn(6.0f, s_gx);
@@ -494,58 +526,10 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
   for (int t = 0; t < 2; ++t)
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[t][i] += acc2[t][i];
-  if (KS > 1 && a.gsplit) {
-    // partial u of this CTA -> the workspace; count in on the group's arrival
-    // word; the last CTA adds the ks partials in K order (deterministic)
-    const int g = (int)(blockIdx.x / KS);
-    float* mine = a.upart + ((size_t)g * KS + kidx) * (size_t)(32 * r);
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int tt = warp + 16 * t;
-      if (tt < n_mma)
-        __stcg(reinterpret_cast<float4*>(mine + (tt * 32 + lane) * 4), make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]));
-    }
-    __threadfence();
-    __syncthreads();
-    __shared__ int last_sh;
-    if (tid == 0) {
-      unsigned long long* w = a.ucnt + g;
-      unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(w), seen;
-      int last = 0;
-      for (;;) {
-        const bool same = (old >> 8) == a.epoch;
-        const unsigned long long cnt = same ? (old & 0xFF) : 0ull;
-        const unsigned long long next = (cnt + 1 == (unsigned long long)KS) ? 0ull : ((a.epoch << 8) | (cnt + 1));
-        seen = atomicCAS(w, old, next);
-        if (seen == old) { last = cnt + 1 == (unsigned long long)KS; break; }
-        old = seen;
-      }
-      last_sh = last;
-    }
-    __syncthreads();
-    if (!last_sh) return;
-    __threadfence();
-    const float* base = a.upart + (size_t)g * KS * (size_t)(32 * r);
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int tt = warp + 16 * t;
-      if (tt < n_mma) {
-        const float4* src = reinterpret_cast<const float4*>(base) + tt * 32 + lane;
-        const size_t step = (size_t)(32 * r) / 4;   // float4s per partial
-        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int k0 = 0; k0 < KS; k0 += 8) {         // eight loads in flight, added in order
-          float4 w[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) w[i] = k0 + i < KS ? __ldcg(src + (size_t)(k0 + i) * step) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            if (k0 + i < KS) { s.x += w[i].x; s.y += w[i].y; s.z += w[i].z; s.w += w[i].w; }
-        }
-        acc[t][0] = s.x; acc[t][1] = s.y; acc[t][2] = s.z; acc[t][3] = s.w;
-      }
-    }
-  } else if (KS > 1) {
-    // partial u of this CTA -> its shared memory; CTA 0 adds ranks 1..ks-1 in order
+  if (KS > 1) {
+    // 1. a cluster's partials -> its CTA 0 through distributed shared memory, in rank order
+    const int CL = GS ? kActClusterKs : KS;   // CTAs per cluster
+    const int crank = kidx % CL;
     float* red = reinterpret_cast<float*>(act_smem);
     __syncthreads();   // the last chunk's MMAs have read their operands
 #pragma unroll
@@ -555,8 +539,8 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
         *reinterpret_cast<float4*>(red + (tt * 32 + lane) * 4) = make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
     }
     cluster_sync();
-    if (kidx == 0) {
-      for (int src = 1; src < KS; ++src) {
+    if (crank == 0) {
+      for (int src = 1; src < CL; ++src) {
         const uint32_t base = mapa_shared(smem_u32(red), (uint32_t)src);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
@@ -569,7 +553,58 @@ __global__ void __launch_bounds__(kActThreads, 1) act_quant_kernel(const ActArgs
       }
     }
     cluster_sync();   // every partial stays in place until CTA 0 has read it
-    if (kidx != 0) return;
+    if (crank != 0) return;
+    if constexpr (GS) {
+      // 2. the ks / 8 cluster sums meet in the workspace: each counts in on the
+      //    group's arrival word; the last one adds them in K order
+      const int g = (int)(blockIdx.x / KS);
+      const int nc = KS / CL, kc = kidx / CL;
+      float* mine = a.upart + ((size_t)g * nc + kc) * (size_t)(32 * r);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int tt = warp + 16 * t;
+        if (tt < n_mma)
+          __stcg(reinterpret_cast<float4*>(mine + (tt * 32 + lane) * 4), make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]));
+      }
+      __threadfence();
+      __syncthreads();
+      __shared__ int last_sh;
+      if (tid == 0) {
+        unsigned long long* w = a.ucnt + g;
+        unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(w), seen;
+        int last = 0;
+        for (;;) {
+          const bool same = (old >> 8) == a.epoch;
+          const unsigned long long cnt = same ? (old & 0xFF) : 0ull;
+          const unsigned long long next = (cnt + 1 == (unsigned long long)nc) ? 0ull : ((a.epoch << 8) | (cnt + 1));
+          seen = atomicCAS(w, old, next);
+          if (seen == old) { last = cnt + 1 == (unsigned long long)nc; break; }
+          old = seen;
+        }
+        last_sh = last;
+      }
+      __syncthreads();
+      if (!last_sh) return;
+      __threadfence();
+      const float* base = a.upart + (size_t)g * nc * (size_t)(32 * r);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int tt = warp + 16 * t;
+        if (tt < n_mma) {
+          const float4* src = reinterpret_cast<const float4*>(base) + tt * 32 + lane;
+          const size_t step = (size_t)(32 * r) / 4;   // float4s per partial
+          float4 w[kActGMaxKs / kActClusterKs];
+#pragma unroll
+          for (int i = 0; i < kActGMaxKs / kActClusterKs; ++i)
+            w[i] = i < nc ? __ldcg(src + (size_t)i * step) : make_float4(0.f, 0.f, 0.f, 0.f);
+          float4 s4 = w[0];
+#pragma unroll
+          for (int i = 1; i < kActGMaxKs / kActClusterKs; ++i)
+            if (i < nc) { s4.x += w[i].x; s4.y += w[i].y; s4.z += w[i].z; s4.w += w[i].w; }
+          acc[t][0] = s4.x; acc[t][1] = s4.y; acc[t][2] = s4.z; acc[t][3] = s4.w;
+        }
+      }
+    }
   }
   // u' = u * inv_alpha, split into bf16 hi + lo: [hi | lo (| hi) | 0 pad];
   // NVFP4 keeps it as swizzled low-rank tiles over the padded rows
@@ -1124,19 +1159,12 @@ constexpr int kEpiWarps = 8;
 constexpr int kP_Threads = 16 * 32;
 constexpr int kEpiChunk = 32 * 128;               // 32 rows x 64 bf16 columns, 128-byte swizzled
 constexpr int kP_Smem = kP_Stages * kS_Size + kEpiWarps * kEpiChunk + 1024;
-// Chained form (the epilogue emits the next layer's quantised input): a
-// 4-deep ring; the tile's X^16 (128 rows x 256 columns bf16, four 64-column
-// swizzled tiles) and this CTA's half of the next layer's L1^T rows for the
-// tile's 256 columns replace the output chunks; the partial down projection
-// (next rank <= 32 columns) sits in TMEM after the scale slots.
-constexpr int kC_Stages = 4;
+// Chained form (the epilogue emits the next layer's quantised input): the
+// same ring; the output chunks' 32 KB hold the next layer's L1 rows of the
+// tile's 256 columns as fp32 ([256][r'], r' <= 32), then the exchange of the
+// two column halves' partial down projections.
 constexpr int kC_MaxR = 32;
-constexpr int kC_XHat = 4 * kLRTile;                      // 65536
-constexpr int kC_L1 = 4 * (kC_MaxR / 2) * 128;            // 8192
-constexpr int kC_Smem = kC_Stages * kS_Size + kC_XHat + kC_L1 + 1024;
-constexpr uint32_t kC_UCol = 256 + 48 * kC_Stages;        // 448
-static_assert(kC_UCol + kC_MaxR <= 512, "TMEM columns");
-static_assert((kC_Stages * kS_Size) % 1024 == 0, "X^16 tiles must start on a 1024-byte boundary");
+static_assert(256 * kC_MaxR * 4 <= kEpiWarps * kEpiChunk, "the L1 slab fits the output chunks");
 
 struct PairArgs {
   int64_t M, Mp;
@@ -1154,6 +1182,7 @@ struct PairArgs {
   float* part;             // ks > 1: fp32 partial sums [ks][M][N]
   int* cnt;                // ks > 1: arrival counters [tiles][16] (zero between calls)
   // chained form only: the next layer's input instead of Y
+  const uint16_t* nx_l1t;       // next layer's L1^T, r' x N bf16
   const float* nx_inv_lambda;   // next layer's 1/lambda (N values)
   const BlobHeader* nx_hdr;     // next layer's header (activation tensor scale)
   uint8_t* nx_atiles;           // next layer's activation tiles [Mp/128][N/256]
@@ -1163,19 +1192,16 @@ struct PairArgs {
 
 template <bool CHAIN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
-    gemm_nvfp4_pair_kernel(const PairArgs g, const __grid_constant__ CUtensorMap tm_y,
-                           const __grid_constant__ CUtensorMap tm_l1n) {
-  constexpr int kStages = CHAIN ? kC_Stages : kP_Stages;
+    gemm_nvfp4_pair_kernel(const PairArgs g, const __grid_constant__ CUtensorMap tm_y) {
+  constexpr int kStages = kP_Stages;
   extern __shared__ __align__(1024) uint8_t gsmem_raw[];
   __shared__ uint64_t landed_bar[kStages], empty_bar[kStages], ready_bar[kStages], accf_bar, acce_bar;
-  __shared__ uint64_t xready_bar, ufull_bar, l1_bar;   // chained form
+  __shared__ uint64_t ep_bar;   // chained form: the eight epilogue warps of this CTA
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ychunks = smem + kStages * kS_Size;   // one 4 KB output chunk per epilogue warp
-  uint8_t* xhat = smem + kStages * kS_Size;      // chained form: X^16 tiles, then the L1^T half
-  uint8_t* l1buf = xhat + kC_XHat;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -1196,9 +1222,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
     }
     mbar_init(&accf_bar, 1);
     mbar_init(&acce_bar, 2 * kEpiWarps);
-    mbar_init(&xready_bar, 2 * kEpiWarps);
-    mbar_init(&ufull_bar, 1);
-    mbar_init(&l1_bar, 1);
+    mbar_init(&ep_bar, kEpiWarps);
     abort_sh = 0;
     fence_mbar_init();
   }
@@ -1258,26 +1282,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
       const uint32_t id_f4 = idesc_nvf4(256, 256);
       int it = 0, tcount = 0;
       bool dead = false;
-      // chained form: tile t's partial down projection X^16 L1 (M = 256, N =
-      // next rank, K = the tile's 256 columns) once its epilogue has staged
-      // X^16 and the L1^T halves in both CTAs; issued after the next tile's
-      // main loop so the tensor pipe never waits for the epilogue
-      const bool down = CHAIN && g.nx_r > 0;
-      auto down_proj = [&](int t) -> bool {
-        if (!mbar_wait_cluster(&xready_bar, (uint32_t)t & 1u, abort_flag)) { give_up_both(); return false; }
-        tc_fence_after();
-        const uint32_t id_u = idesc_f16_bf16(256, g.nx_r);
-        const uint32_t xa = smem_u32(xhat), la = smem_u32(l1buf);
-        const uint32_t lc = (uint32_t)(g.nx_r / 2) * 128u;   // bytes of one 64-column L1^T chunk
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            mma_f16_pair(tbase + kC_UCol, desc_k_sw128(xa + c * kLRTile + 32 * q), desc_k_sw128(la + c * lc + 32 * q),
-                         id_u, (c | q) != 0);
-        mma_commit_pair(&ufull_bar, 0x3);
-        return true;
-      };
       for (int item = pair; item < num_items && !dead; item += pairs, ++tcount) {
         const int lr = item_lr(item);
         if (!mbar_wait(&acce_bar, (tcount & 1) ^ 1, abort_flag)) { give_up_both(); break; }
@@ -1303,10 +1307,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
           }
           mma_commit_pair(&empty_bar[s], 0x3);
         }
-        if (down && !dead && tcount > 0 && !down_proj(tcount - 1)) dead = true;
         if (!dead) mma_commit_pair(&accf_bar, 0x3);
       }
-      if (down && !dead && tcount > 0) down_proj(tcount - 1);
       if (*abort_flag) {
         mma_commit_pair(&accf_bar, 0x3);
         mbar_drain(&accf_bar, tcount & 1);
@@ -1359,6 +1361,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
     const float alpha = g.hdr->s_gx * g.hdr->s_gw;
     uint8_t* ybuf = ychunks + (warp - 8) * kEpiChunk;
     int tcount = 0;
+    int ep_phase = 0;   // uses of ep_bar so far (chained form)
     for (int item = pair; item < num_items; item += pairs, ++tcount) {
       const int tile = item / g.ks, kq = item % g.ks;
       const int mt = tile / n_tiles, nt = tile % n_tiles;
@@ -1366,16 +1369,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
       float bl[4];   // bias of columns col0 + 32 j + lane
 #pragma unroll
       for (int j = 0; j < 4; ++j) bl[j] = __ldg(g.bias + col0 + 32 * j + lane);
-      if (CHAIN && g.nx_r > 0 && warp == 8 && lane == 0) {
-        // this CTA's half of the next layer's L1^T rows, the tile's 256
-        // columns (the buffer is free: the previous tile's down projection
-        // completed before this warp read its result)
-        const int rh = g.nx_r / 2;
-        mbar_arrive_expect_tx(&l1_bar, (uint32_t)(256 * g.nx_r));
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          tma_load_2d(l1buf + c * rh * 128, &tm_l1n, &l1_bar, nt * 256 + 64 * c, (int)rank * rh);
-      }
       if (!mbar_wait(&accf_bar, tcount & 1, abort_flag)) { give_up_both(); break; }
       tc_fence_after();
       uint32_t v[128];
@@ -1392,16 +1385,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
         // The next layer's input, as its activation kernel would make it from
         // this layer's bf16 output y: x^ = fp32(y) * inv_lambda', one NVFP4
         // block per 16 columns (codes and E4M3 scale into the next layer's
-        // activation tile (row tile, K slab nt)), and X^16 = bf16(x^) staged
-        // for the partial down projection.  Rows past M quantise zeros.
+        // activation tile (row tile, K slab nt)), and this tile's share of
+        // the down projection u' += X^16 L1' (X^16 = bf16(x^)) on the CUDA
+        // cores, two fp32 lanes per instruction, columns in order.  Rows past
+        // M quantise zeros.
         const int rl = q * 32 + lane;                     // row inside this CTA's 128
+        const int et = (warp - 8) * 32 + lane;            // 0..255: the tile column this thread stages
         const bool live = row0 + lane < g.M;
+        const int rn = g.nx_r;
+        float* l1s = reinterpret_cast<float*>(ychunks);   // [256][rn] fp32, then [128][rn] exchange
+        // y = bf16(alpha acc + b), two per register (frees the fp32 accumulator copy)
+        uint32_t yb[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const int e = 2 * i;
+          const float b0 = __shfl_sync(0xffffffffu, bl[e >> 5], e & 31);
+          const float b1 = __shfl_sync(0xffffffffu, bl[(e + 1) >> 5], (e + 1) & 31);
+          yb[i] = (uint32_t)bf16_rn(fmaf(alpha, __uint_as_float(v[e]), b0)) |
+                  ((uint32_t)bf16_rn(fmaf(alpha, __uint_as_float(v[e + 1]), b1)) << 16);
+        }
+        // epilogue-wide hand-offs (the 8 epilogue warps of this CTA), bounded waits
+        auto ep_sync = [&]() -> bool {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ep_bar);
+          const bool ok = mbar_wait(&ep_bar, (uint32_t)(ep_phase & 1), abort_flag);
+          ++ep_phase;
+          return __all_sync(0xffffffffu, ok);
+        };
+        if (rn > 0) {
+          // the slab area is free (every warp is past the previous tile's
+          // exchange): this thread's column of L1'^T for the tile -> fp32 row
+          if (!ep_sync()) { give_up_both(); break; }
+          const uint16_t* src = g.nx_l1t + (size_t)nt * 256 + et;
+#pragma unroll
+          for (int k4 = 0; k4 < kC_MaxR / 4; ++k4) {
+            if (4 * k4 < rn) {
+              float w[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) w[j] = __uint_as_float((uint32_t)__ldg(src + (size_t)(4 * k4 + j) * g.N) << 16);
+              reinterpret_cast<float4*>(l1s + (size_t)et * rn)[k4] = make_float4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+        if (rn > 0 && !ep_sync()) { give_up_both(); break; }   // the slab is complete
         const float s_gx = g.nx_hdr->s_gx;
         const float six_sg = __fmul_rn(6.0f, s_gx);
         const float r6 = recip_ok(six_sg) ? __frcp_rn(six_sg) : 0.0f;
         uint8_t* ntile = g.nx_atiles + ((size_t)(2 * mt + (int)rank) * (size_t)n_tiles + (size_t)nt) * kATile;
         const float4* il4 = reinterpret_cast<const float4*>(g.nx_inv_lambda + col0);
-        uint32_t sc = 0, cw[4];
+        uint32_t sc = 0, cw[4], x16[64];
 #pragma unroll
         for (int b = 0; b < 8; ++b) {                     // block b: columns 16 b .. 16 b + 15 of this half
           float xh[16];
@@ -1412,8 +1444,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int e = 16 * b + 4 * j4 + j;
-              const float bb = __shfl_sync(0xffffffffu, bl[e >> 5], e & 31);
-              const float yv = __uint_as_float((uint32_t)bf16_rn(fmaf(alpha, __uint_as_float(v[e]), bb)) << 16);
+              const uint32_t pr = yb[e >> 1];
+              const float yv = __uint_as_float((e & 1) ? (pr & 0xFFFF0000u) : (pr << 16));
               xh[4 * j4 + j] = live ? __fmul_rn(yv, ilv[j]) : 0.0f;
             }
           }
@@ -1430,53 +1462,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
                                          (rl >> 5) * 4) = sc;
             sc = 0;
           }
-          if (g.nx_r > 0) {   // X^16 of the block: two 16-byte pieces of its 64-column tile
-            uint32_t x16[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              x16[i] = (uint32_t)bf16_rn(xh[2 * i]) | ((uint32_t)bf16_rn(xh[2 * i + 1]) << 16);
-            uint8_t* xt = xhat + (2 * h + (b >> 2)) * kLRTile + rl * 128;
-            const int p0 = 2 * (b & 3);
-            *reinterpret_cast<uint4*>(xt + ((p0 ^ (rl & 7)) << 4)) = make_uint4(x16[0], x16[1], x16[2], x16[3]);
-            *reinterpret_cast<uint4*>(xt + (((p0 + 1) ^ (rl & 7)) << 4)) = make_uint4(x16[4], x16[5], x16[6], x16[7]);
-          }
+          for (int i = 0; i < 8; ++i)
+            x16[8 * b + i] = (uint32_t)bf16_rn(xh[2 * i]) | ((uint32_t)bf16_rn(xh[2 * i + 1]) << 16);
         }
-        if (g.nx_r > 0) {
-          // hand X^16 (and, from warp 8, the landed L1^T half) to the MMA
-          // thread, then take this tile's partial down projection: lane
-          // quarter q, columns [h r/2, (h + 1) r/2) of the next rank
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            if (warp == 8 && !mbar_wait(&l1_bar, tcount & 1, abort_flag)) give_up_both();
-            mbar_arrive_cluster_release(mapa_shared(smem_u32(&xready_bar), 0));
-          }
-          __syncwarp();
-          if (!mbar_wait(&ufull_bar, tcount & 1, abort_flag)) { give_up_both(); break; }
-          tc_fence_after();
-          const int rh = g.nx_r / 2;
-          const uint32_t ua = tbase + ((uint32_t)(q * 32) << 16) + kC_UCol + (uint32_t)(h * rh);
-          float* dst = g.nx_upart + ((size_t)nt * (size_t)g.Mp + (size_t)(row0 + lane)) * g.nx_r + h * rh;
-          if (rh == 16) {
-            uint32_t uv[16];
-            tmem_ld_16cols(ua, uv);
-            tmem_ld_wait();
+        if (rn > 0) {
+          // u' += X^16 L1' over this half's 128 columns, in column order
+          uint64_t u2[kC_MaxR / 2];
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-              reinterpret_cast<float4*>(dst)[c] =
-                  make_float4(__uint_as_float(uv[4 * c]), __uint_as_float(uv[4 * c + 1]),
-                              __uint_as_float(uv[4 * c + 2]), __uint_as_float(uv[4 * c + 3]));
-          } else {
-            uint32_t uv[8];
-            tmem_ld_8cols(ua, uv);
-            tmem_ld_wait();
+          for (int k = 0; k < kC_MaxR / 2; ++k) u2[k] = 0ull;
+          // a column pair per iteration (x16 is read from the thread's local
+          // copy: one 32-bit load per two columns beside 2 x 8 shared loads)
+#pragma unroll 1
+          for (int c2 = 0; c2 < 64; ++c2) {
+            const uint32_t pr = x16[c2];
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
-              reinterpret_cast<float4*>(dst)[c] =
-                  make_float4(__uint_as_float(uv[4 * c]), __uint_as_float(uv[4 * c + 1]),
-                              __uint_as_float(uv[4 * c + 2]), __uint_as_float(uv[4 * c + 3]));
+            for (int hl = 0; hl < 2; ++hl) {
+              const float xv = __uint_as_float(hl ? (pr & 0xFFFF0000u) : (pr << 16));
+              const uint64_t x2 = f2_pack(xv, xv);
+              const ulonglong2* w = reinterpret_cast<const ulonglong2*>(l1s + (size_t)(h * 128 + 2 * c2 + hl) * rn);
+#pragma unroll
+              for (int k4 = 0; k4 < kC_MaxR / 4; ++k4) {
+                if (4 * k4 < rn) {
+                  const ulonglong2 ww = w[k4];
+                  u2[2 * k4] = f2_fma(x2, ww.x, u2[2 * k4]);
+                  u2[2 * k4 + 1] = f2_fma(x2, ww.y, u2[2 * k4 + 1]);
+                }
+              }
+            }
           }
-          tc_fence_before();
+          // the two column halves of a row meet: half 1 parks its partial in the
+          // slab area, half 0 adds it (in that order) and stores the tile's partial
+          if (!ep_sync()) { give_up_both(); break; }      // every warp is done with the slab
+          ulonglong2* xch = reinterpret_cast<ulonglong2*>(l1s + (size_t)rl * rn);
+          if (h == 1) {
+#pragma unroll
+            for (int k4 = 0; k4 < kC_MaxR / 4; ++k4)
+              if (4 * k4 < rn) xch[k4] = make_ulonglong2(u2[2 * k4], u2[2 * k4 + 1]);
+          }
+          if (!ep_sync()) { give_up_both(); break; }
+          if (h == 0) {
+            float4* dst = reinterpret_cast<float4*>(g.nx_upart + ((size_t)nt * (size_t)g.Mp + (size_t)(row0 + lane)) * rn);
+#pragma unroll
+            for (int k4 = 0; k4 < kC_MaxR / 4; ++k4) {
+              if (4 * k4 < rn) {
+                const ulonglong2 o = xch[k4];
+                float a0, a1, a2, a3, b0, b1, b2, b3;
+                f2_unpack(u2[2 * k4], a0, a1); f2_unpack(u2[2 * k4 + 1], a2, a3);
+                f2_unpack(o.x, b0, b1); f2_unpack(o.y, b2, b3);
+                __stcg(dst + k4, make_float4(a0 + b0, a1 + b1, a2 + b2, a3 + b3));
+              }
+            }
+          }
         }
         continue;
       }
@@ -2363,7 +2400,7 @@ svdq_status device_ready() {
       d.ok = cudaFuncSetAttribute(dev::gemm_nvfp4_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   dev::kP_Smem) == cudaSuccess &&
              cudaFuncSetAttribute(dev::gemm_nvfp4_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  dev::kC_Smem) == cudaSuccess &&
+                                  dev::kP_Smem) == cudaSuccess &&
              cudaFuncSetAttribute(dev::gemm_nvfp4_small_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   dev::sm_smem(16)) == cudaSuccess &&
              cudaFuncSetAttribute(dev::gemm_nvfp4_small_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -2374,13 +2411,17 @@ svdq_status device_ready() {
                                   i4_smem) == cudaSuccess;
       const int act_smem = dev::kActSmemMax;
       d.ok = d.ok &&
-             cudaFuncSetAttribute(dev::act_quant_kernel<SVDQ_NVFP4, SVDQ_BF16>,
+             cudaFuncSetAttribute(dev::act_quant_kernel<SVDQ_NVFP4, SVDQ_BF16, false>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, act_smem) == cudaSuccess &&
-             cudaFuncSetAttribute(dev::act_quant_kernel<SVDQ_NVFP4, SVDQ_F16>,
+             cudaFuncSetAttribute(dev::act_quant_kernel<SVDQ_NVFP4, SVDQ_F16, false>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, act_smem) == cudaSuccess &&
-             cudaFuncSetAttribute(dev::act_quant_kernel<SVDQ_INT4_G64, SVDQ_BF16>,
+             cudaFuncSetAttribute(dev::act_quant_kernel<SVDQ_NVFP4, SVDQ_BF16, true>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, act_smem) == cudaSuccess &&
-             cudaFuncSetAttribute(dev::act_quant_kernel<SVDQ_INT4_G64, SVDQ_F16>,
+             cudaFuncSetAttribute(dev::act_quant_kernel<SVDQ_NVFP4, SVDQ_F16, true>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, act_smem) == cudaSuccess &&
+             cudaFuncSetAttribute(dev::act_quant_kernel<SVDQ_INT4_G64, SVDQ_BF16, false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, act_smem) == cudaSuccess &&
+             cudaFuncSetAttribute(dev::act_quant_kernel<SVDQ_INT4_G64, SVDQ_F16, false>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, act_smem) == cudaSuccess &&
              cudaFuncSetAttribute(dev::act_nvfp4_kernel<SVDQ_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   dev::kAN_Budget) == cudaSuccess &&
@@ -2429,21 +2470,27 @@ std::atomic<unsigned long long> g_act_epoch{
 template <int FMT>
 cudaError_t launch_act(const svdq_params* p, dev::ActArgs a, int64_t Mp, cudaStream_t stream) {
   a.ks = act_k_split(Mp, p->K);
-  a.gsplit = 0;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(dev::kActThreads);
   cfg.stream = stream;
-  if (FMT == SVDQ_NVFP4 && a.upart != nullptr) {
+  if constexpr (FMT == SVDQ_NVFP4) if (a.upart != nullptr) {
     // few live 32-token groups: only they run (rows past them are never read
-    // for live tokens), ks > 8 CTAs each, partials through the workspace
+    // for live tokens), ks > 8 CTAs each as clusters of 8; the clusters'
+    // partials meet in the workspace
     a.ks = act_small_ks(a.M, p->K);
-    a.gsplit = 1;
     a.epoch = g_act_epoch.fetch_add(1) & 0x00FFFFFFFFFFFFFFull;
     if (a.epoch == 0) a.epoch = g_act_epoch.fetch_add(1) & 0x00FFFFFFFFFFFFFFull;
     cfg.gridDim = dim3((unsigned)((a.M + dev::kActRows - 1) / dev::kActRows * a.ks));
     cfg.dynamicSmemBytes = (size_t)dev::act_smem_bytes(p->rank, p->K / a.ks);
-    if (p->act_dtype == SVDQ_BF16) return cudaLaunchKernelEx(&cfg, dev::act_quant_kernel<FMT, SVDQ_BF16>, a);
-    return cudaLaunchKernelEx(&cfg, dev::act_quant_kernel<FMT, SVDQ_F16>, a);
+    cudaLaunchAttribute cat[1];
+    cat[0].id = cudaLaunchAttributeClusterDimension;
+    cat[0].val.clusterDim.x = (unsigned)kActClusterKs;
+    cat[0].val.clusterDim.y = 1;
+    cat[0].val.clusterDim.z = 1;
+    cfg.attrs = cat;
+    cfg.numAttrs = 1;
+    if (p->act_dtype == SVDQ_BF16) return cudaLaunchKernelEx(&cfg, dev::act_quant_kernel<FMT, SVDQ_BF16, true>, a);
+    return cudaLaunchKernelEx(&cfg, dev::act_quant_kernel<FMT, SVDQ_F16, true>, a);
   }
   cfg.gridDim = dim3((unsigned)(Mp / dev::kActRows * a.ks));
   cfg.dynamicSmemBytes = (size_t)dev::act_smem_bytes(p->rank, p->K / a.ks);
@@ -2454,8 +2501,8 @@ cudaError_t launch_act(const svdq_params* p, dev::ActArgs a, int64_t Mp, cudaStr
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  if (p->act_dtype == SVDQ_BF16) return cudaLaunchKernelEx(&cfg, dev::act_quant_kernel<FMT, SVDQ_BF16>, a);
-  return cudaLaunchKernelEx(&cfg, dev::act_quant_kernel<FMT, SVDQ_F16>, a);
+  if (p->act_dtype == SVDQ_BF16) return cudaLaunchKernelEx(&cfg, dev::act_quant_kernel<FMT, SVDQ_BF16, false>, a);
+  return cudaLaunchKernelEx(&cfg, dev::act_quant_kernel<FMT, SVDQ_F16, false>, a);
 }
 
 }  // namespace
@@ -2494,7 +2541,6 @@ svdq_status launch_quantize(const svdq_params* p, const void* blob_dev, const vo
   const bool gsplit = p->fmt == SVDQ_NVFP4 && M <= 256 && W.off_ucnt > W.off_upart;
   a.upart = gsplit ? reinterpret_cast<float*>(ws + W.off_upart) : nullptr;
   a.ucnt = gsplit ? reinterpret_cast<unsigned long long*>(ws + W.off_ucnt) : nullptr;
-  a.gsplit = 0;
   a.epoch = 0;
   // NVFP4 above 256 tokens: the 128-token-tile kernel (tcgen05 down projection).
   // Up to 256 tokens the 32-token kernel wins: its latency chain per call is
@@ -2617,7 +2663,7 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_pair_kernel<false>, g, tm_y, tm_y);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_pair_kernel<false>, g, tm_y);
     if (e != cudaSuccess) return cuda_fail(e, "gemm_nvfp4_pair_kernel launch");
     return launch_status("gemm_nvfp4_pair_kernel launch");
   }
@@ -2701,23 +2747,21 @@ svdq_status launch_gemm_chain(const svdq_params* p, const void* blob_dev, int64_
   g.nx_atiles = wsn + Wn.off_xq;
   g.nx_upart = reinterpret_cast<float*>(ws + C.off_extra);
   g.nx_r = rn;
-  CUtensorMap tm_l1n{};
-  if (rn > 0 && !make_map(&tm_l1n, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, nblob + Bn.off_l1t, (uint64_t)N, (uint64_t)rn,
-                          (uint64_t)N * 2, 64, (uint32_t)(rn / 2)))
-    return cuda_fail(cudaErrorInvalidValue, "tensor map encode (next layer L1)");
+  g.nx_l1t = reinterpret_cast<const uint16_t*>(nblob + Bn.off_l1t);
+  const CUtensorMap unused_map{};   // the chained form writes no Y
   const int tiles = (N / 256) * (int)(W.Mp / 256);
   const int pairs = std::max(1, std::min(tiles, num_sms() / 2));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
   cfg.blockDim = dim3(dev::kP_Threads);
-  cfg.dynamicSmemBytes = dev::kC_Smem;
+  cfg.dynamicSmemBytes = dev::kP_Smem;
   cfg.stream = stream;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_pair_kernel<true>, g, tm_l1n, tm_l1n);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_pair_kernel<true>, g, unused_map);
   if (e != cudaSuccess) return cuda_fail(e, "gemm_nvfp4_pair_kernel (chained) launch");
   if (rn > 0) {
     const int lrw_n = lr_width(*pn);

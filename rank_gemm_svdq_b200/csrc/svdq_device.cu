@@ -1159,12 +1159,19 @@ constexpr int kEpiWarps = 8;
 constexpr int kP_Threads = 16 * 32;
 constexpr int kEpiChunk = 32 * 128;               // 32 rows x 64 bf16 columns, 128-byte swizzled
 constexpr int kP_Smem = kP_Stages * kS_Size + kEpiWarps * kEpiChunk + 1024;
-// Chained form (the epilogue emits the next layer's quantised input): the
-// same ring; the output chunks' 32 KB hold the next layer's L1 rows of the
-// tile's 256 columns as fp32 ([256][r'], r' <= 32), then the exchange of the
-// two column halves' partial down projections.
+// Chained form (the epilogue emits the next layer's quantised input): a
+// 4-deep ring; the tile's X^16 (128 rows x 256 columns bf16, four 64-column
+// swizzled tiles) and this CTA's half of the next layer's L1^T rows for the
+// tile's 256 columns replace the output chunks; the partial down projection
+// (next rank <= 32 columns) sits in TMEM after the scale slots.
+constexpr int kC_Stages = 4;
 constexpr int kC_MaxR = 32;
-static_assert(256 * kC_MaxR * 4 <= kEpiWarps * kEpiChunk, "the L1 slab fits the output chunks");
+constexpr int kC_XHat = 4 * kLRTile;                      // 65536
+constexpr int kC_L1 = 4 * (kC_MaxR / 2) * 128;            // 8192
+constexpr int kC_Smem = kC_Stages * kS_Size + kC_XHat + kC_L1 + 1024;
+constexpr uint32_t kC_UCol = 256 + 48 * kC_Stages;        // 448
+static_assert(kC_UCol + kC_MaxR <= 512, "TMEM columns");
+static_assert((kC_Stages * kS_Size) % 1024 == 0, "X^16 tiles must start on a 1024-byte boundary");
 
 struct PairArgs {
   int64_t M, Mp;
@@ -1182,7 +1189,6 @@ struct PairArgs {
   float* part;             // ks > 1: fp32 partial sums [ks][M][N]
   int* cnt;                // ks > 1: arrival counters [tiles][16] (zero between calls)
   // chained form only: the next layer's input instead of Y
-  const uint16_t* nx_l1t;       // next layer's L1^T, r' x N bf16
   const float* nx_inv_lambda;   // next layer's 1/lambda (N values)
   const BlobHeader* nx_hdr;     // next layer's header (activation tensor scale)
   uint8_t* nx_atiles;           // next layer's activation tiles [Mp/128][N/256]
@@ -1192,16 +1198,19 @@ struct PairArgs {
 
 template <bool CHAIN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
-    gemm_nvfp4_pair_kernel(const PairArgs g, const __grid_constant__ CUtensorMap tm_y) {
-  constexpr int kStages = kP_Stages;
+    gemm_nvfp4_pair_kernel(const PairArgs g, const __grid_constant__ CUtensorMap tm_y,
+                           const __grid_constant__ CUtensorMap tm_l1n) {
+  constexpr int kStages = CHAIN ? kC_Stages : kP_Stages;
   extern __shared__ __align__(1024) uint8_t gsmem_raw[];
   __shared__ uint64_t landed_bar[kStages], empty_bar[kStages], ready_bar[kStages], accf_bar, acce_bar;
-  __shared__ uint64_t ep_bar;   // chained form: the eight epilogue warps of this CTA
+  __shared__ uint64_t xready_bar, ufull_bar, l1_bar;   // chained form
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ychunks = smem + kStages * kS_Size;   // one 4 KB output chunk per epilogue warp
+  uint8_t* xhat = smem + kStages * kS_Size;      // chained form: X^16 tiles, then the L1^T half
+  uint8_t* l1buf = xhat + kC_XHat;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -1222,7 +1231,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
     }
     mbar_init(&accf_bar, 1);
     mbar_init(&acce_bar, 2 * kEpiWarps);
-    mbar_init(&ep_bar, kEpiWarps);
+    mbar_init(&xready_bar, 2 * kEpiWarps);
+    mbar_init(&ufull_bar, 1);
+    mbar_init(&l1_bar, 1);
     abort_sh = 0;
     fence_mbar_init();
   }
@@ -1282,12 +1293,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
       const uint32_t id_f4 = idesc_nvf4(256, 256);
       int it = 0, tcount = 0;
       bool dead = false;
+      // chained form: tile t's partial down projection X^16 L1 (M = 256, N =
+      // next rank, K = the tile's 256 columns) once its epilogue has staged
+      // X^16 and the L1^T halves in both CTAs: between the stages of the next
+      // tile's main loop as soon as the hand-off has landed (polled, never
+      // waited on there), else at that loop's end
+      const bool down = CHAIN && g.nx_r > 0;
+      int pend = -1;   // the tile whose down projection is still to be issued
+      auto issue_down = [&](int t) {
+        tc_fence_after();
+        const uint32_t id_u = idesc_f16_bf16(256, g.nx_r);
+        const uint32_t xa = smem_u32(xhat), la = smem_u32(l1buf);
+        const uint32_t lc = (uint32_t)(g.nx_r / 2) * 128u;   // bytes of one 64-column L1^T chunk
+#pragma unroll 1
+        for (int cq = 0; cq < 16; ++cq) {   // 64-column chunk cq / 4, K step cq % 4 (a loop: this warp has 56 registers)
+          const int c = cq >> 2, q = cq & 3;
+          mma_f16_pair(tbase + kC_UCol, desc_k_sw128(xa + c * kLRTile + 32 * q), desc_k_sw128(la + c * lc + 32 * q),
+                       id_u, cq != 0);
+        }
+        mma_commit_pair(&ufull_bar, 0x3);
+        pend = -1;
+      };
+      // blocking form (end of a main loop, or after the last tile)
+      auto down_proj = [&](int t) -> bool {
+        if (!mbar_wait_cluster(&xready_bar, (uint32_t)t & 1u, abort_flag)) { give_up_both(); return false; }
+        issue_down(t);
+        return true;
+      };
       for (int item = pair; item < num_items && !dead; item += pairs, ++tcount) {
         const int lr = item_lr(item);
         if (!mbar_wait(&acce_bar, (tcount & 1) ^ 1, abort_flag)) { give_up_both(); break; }
         tc_fence_after();
+        if (down && tcount > 0) pend = tcount - 1;
         for (int j = 0; j < lr + cpk; ++j, ++it) {
           const int s = it % kStages;
+          // the previous tile's down projection as soon as its epilogue has staged X^16
+          if (pend >= 0 && mbar_try_wait_cluster(&xready_bar, (uint32_t)pend & 1u)) issue_down(pend);
           if (!mbar_wait(&ready_bar[s], (it / kStages) & 1, abort_flag)) { give_up_both(); dead = true; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * kS_Size);
@@ -1307,8 +1348,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
           }
           mma_commit_pair(&empty_bar[s], 0x3);
         }
+        if (!dead && pend >= 0 && !down_proj(pend)) dead = true;
         if (!dead) mma_commit_pair(&accf_bar, 0x3);
       }
+      if (down && !dead && tcount > 0) down_proj(tcount - 1);
       if (*abort_flag) {
         mma_commit_pair(&accf_bar, 0x3);
         mbar_drain(&accf_bar, tcount & 1);
@@ -1361,7 +1404,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
     const float alpha = g.hdr->s_gx * g.hdr->s_gw;
     uint8_t* ybuf = ychunks + (warp - 8) * kEpiChunk;
     int tcount = 0;
-    int ep_phase = 0;   // uses of ep_bar so far (chained form)
     for (int item = pair; item < num_items; item += pairs, ++tcount) {
       const int tile = item / g.ks, kq = item % g.ks;
       const int mt = tile / n_tiles, nt = tile % n_tiles;
@@ -1369,6 +1411,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
       float bl[4];   // bias of columns col0 + 32 j + lane
 #pragma unroll
       for (int j = 0; j < 4; ++j) bl[j] = __ldg(g.bias + col0 + 32 * j + lane);
+      if (CHAIN && g.nx_r > 0 && warp == 8 && lane == 0) {
+        // this CTA's half of the next layer's L1^T rows, the tile's 256
+        // columns (the buffer is free: the previous tile's down projection
+        // completed before this warp read its result)
+        const int rh = g.nx_r / 2;
+        mbar_arrive_expect_tx(&l1_bar, (uint32_t)(256 * g.nx_r));
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tma_load_2d(l1buf + c * rh * 128, &tm_l1n, &l1_bar, nt * 256 + 64 * c, (int)rank * rh);
+      }
       if (!mbar_wait(&accf_bar, tcount & 1, abort_flag)) { give_up_both(); break; }
       tc_fence_after();
       uint32_t v[128];
@@ -1385,55 +1437,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
         // The next layer's input, as its activation kernel would make it from
         // this layer's bf16 output y: x^ = fp32(y) * inv_lambda', one NVFP4
         // block per 16 columns (codes and E4M3 scale into the next layer's
-        // activation tile (row tile, K slab nt)), and this tile's share of
-        // the down projection u' += X^16 L1' (X^16 = bf16(x^)) on the CUDA
-        // cores, two fp32 lanes per instruction, columns in order.  Rows past
-        // M quantise zeros.
+        // activation tile (row tile, K slab nt)), and X^16 = bf16(x^) staged
+        // for the partial down projection.  Rows past M quantise zeros.
         const int rl = q * 32 + lane;                     // row inside this CTA's 128
-        const int et = (warp - 8) * 32 + lane;            // 0..255: the tile column this thread stages
         const bool live = row0 + lane < g.M;
-        const int rn = g.nx_r;
-        float* l1s = reinterpret_cast<float*>(ychunks);   // [256][rn] fp32, then [128][rn] exchange
-        // y = bf16(alpha acc + b), two per register (frees the fp32 accumulator copy)
-        uint32_t yb[64];
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const int e = 2 * i;
-          const float b0 = __shfl_sync(0xffffffffu, bl[e >> 5], e & 31);
-          const float b1 = __shfl_sync(0xffffffffu, bl[(e + 1) >> 5], (e + 1) & 31);
-          yb[i] = (uint32_t)bf16_rn(fmaf(alpha, __uint_as_float(v[e]), b0)) |
-                  ((uint32_t)bf16_rn(fmaf(alpha, __uint_as_float(v[e + 1]), b1)) << 16);
-        }
-        // epilogue-wide hand-offs (the 8 epilogue warps of this CTA), bounded waits
-        auto ep_sync = [&]() -> bool {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ep_bar);
-          const bool ok = mbar_wait(&ep_bar, (uint32_t)(ep_phase & 1), abort_flag);
-          ++ep_phase;
-          return __all_sync(0xffffffffu, ok);
-        };
-        if (rn > 0) {
-          // the slab area is free (every warp is past the previous tile's
-          // exchange): this thread's column of L1'^T for the tile -> fp32 row
-          if (!ep_sync()) { give_up_both(); break; }
-          const uint16_t* src = g.nx_l1t + (size_t)nt * 256 + et;
-#pragma unroll
-          for (int k4 = 0; k4 < kC_MaxR / 4; ++k4) {
-            if (4 * k4 < rn) {
-              float w[4];
-#pragma unroll
-              for (int j = 0; j < 4; ++j) w[j] = __uint_as_float((uint32_t)__ldg(src + (size_t)(4 * k4 + j) * g.N) << 16);
-              reinterpret_cast<float4*>(l1s + (size_t)et * rn)[k4] = make_float4(w[0], w[1], w[2], w[3]);
-            }
-          }
-        }
-        if (rn > 0 && !ep_sync()) { give_up_both(); break; }   // the slab is complete
         const float s_gx = g.nx_hdr->s_gx;
         const float six_sg = __fmul_rn(6.0f, s_gx);
         const float r6 = recip_ok(six_sg) ? __frcp_rn(six_sg) : 0.0f;
         uint8_t* ntile = g.nx_atiles + ((size_t)(2 * mt + (int)rank) * (size_t)n_tiles + (size_t)nt) * kATile;
         const float4* il4 = reinterpret_cast<const float4*>(g.nx_inv_lambda + col0);
-        uint32_t sc = 0, cw[4], x16[64];
+        uint32_t sc = 0, cw[4];
 #pragma unroll
         for (int b = 0; b < 8; ++b) {                     // block b: columns 16 b .. 16 b + 15 of this half
           float xh[16];
@@ -1444,8 +1457,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int e = 16 * b + 4 * j4 + j;
-              const uint32_t pr = yb[e >> 1];
-              const float yv = __uint_as_float((e & 1) ? (pr & 0xFFFF0000u) : (pr << 16));
+              const float bb = __shfl_sync(0xffffffffu, bl[e >> 5], e & 31);
+              const float yv = __uint_as_float((uint32_t)bf16_rn(fmaf(alpha, __uint_as_float(v[e]), bb)) << 16);
               xh[4 * j4 + j] = live ? __fmul_rn(yv, ilv[j]) : 0.0f;
             }
           }
@@ -1462,58 +1475,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kP_Threads, 1)
                                          (rl >> 5) * 4) = sc;
             sc = 0;
           }
+          if (g.nx_r > 0) {   // X^16 of the block: two 16-byte pieces of its 64-column tile
+            uint32_t x16[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            x16[8 * b + i] = (uint32_t)bf16_rn(xh[2 * i]) | ((uint32_t)bf16_rn(xh[2 * i + 1]) << 16);
+            for (int i = 0; i < 8; ++i)
+              x16[i] = (uint32_t)bf16_rn(xh[2 * i]) | ((uint32_t)bf16_rn(xh[2 * i + 1]) << 16);
+            uint8_t* xt = xhat + (2 * h + (b >> 2)) * kLRTile + rl * 128;
+            const int p0 = 2 * (b & 3);
+            *reinterpret_cast<uint4*>(xt + ((p0 ^ (rl & 7)) << 4)) = make_uint4(x16[0], x16[1], x16[2], x16[3]);
+            *reinterpret_cast<uint4*>(xt + (((p0 + 1) ^ (rl & 7)) << 4)) = make_uint4(x16[4], x16[5], x16[6], x16[7]);
+          }
         }
-        if (rn > 0) {
-          // u' += X^16 L1' over this half's 128 columns, in column order
-          uint64_t u2[kC_MaxR / 2];
-#pragma unroll
-          for (int k = 0; k < kC_MaxR / 2; ++k) u2[k] = 0ull;
-          // a column pair per iteration (x16 is read from the thread's local
-          // copy: one 32-bit load per two columns beside 2 x 8 shared loads)
-#pragma unroll 1
-          for (int c2 = 0; c2 < 64; ++c2) {
-            const uint32_t pr = x16[c2];
-#pragma unroll
-            for (int hl = 0; hl < 2; ++hl) {
-              const float xv = __uint_as_float(hl ? (pr & 0xFFFF0000u) : (pr << 16));
-              const uint64_t x2 = f2_pack(xv, xv);
-              const ulonglong2* w = reinterpret_cast<const ulonglong2*>(l1s + (size_t)(h * 128 + 2 * c2 + hl) * rn);
-#pragma unroll
-              for (int k4 = 0; k4 < kC_MaxR / 4; ++k4) {
-                if (4 * k4 < rn) {
-                  const ulonglong2 ww = w[k4];
-                  u2[2 * k4] = f2_fma(x2, ww.x, u2[2 * k4]);
-                  u2[2 * k4 + 1] = f2_fma(x2, ww.y, u2[2 * k4 + 1]);
-                }
-              }
-            }
+        if (g.nx_r > 0) {
+          // hand X^16 (and, from warp 8, the landed L1^T half) to the MMA
+          // thread, then take this tile's partial down projection: lane
+          // quarter q, columns [h r/2, (h + 1) r/2) of the next rank
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (warp == 8 && !mbar_wait(&l1_bar, tcount & 1, abort_flag)) give_up_both();
+            mbar_arrive_cluster_release(mapa_shared(smem_u32(&xready_bar), 0));
           }
-          // the two column halves of a row meet: half 1 parks its partial in the
-          // slab area, half 0 adds it (in that order) and stores the tile's partial
-          if (!ep_sync()) { give_up_both(); break; }      // every warp is done with the slab
-          ulonglong2* xch = reinterpret_cast<ulonglong2*>(l1s + (size_t)rl * rn);
-          if (h == 1) {
+          __syncwarp();
+          if (!mbar_wait(&ufull_bar, tcount & 1, abort_flag)) { give_up_both(); break; }
+          tc_fence_after();
+          const int rh = g.nx_r / 2;
+          const uint32_t ua = tbase + ((uint32_t)(q * 32) << 16) + kC_UCol + (uint32_t)(h * rh);
+          float* dst = g.nx_upart + ((size_t)nt * (size_t)g.Mp + (size_t)(row0 + lane)) * g.nx_r + h * rh;
+          if (rh == 16) {
+            uint32_t uv[16];
+            tmem_ld_16cols(ua, uv);
+            tmem_ld_wait();
 #pragma unroll
-            for (int k4 = 0; k4 < kC_MaxR / 4; ++k4)
-              if (4 * k4 < rn) xch[k4] = make_ulonglong2(u2[2 * k4], u2[2 * k4 + 1]);
-          }
-          if (!ep_sync()) { give_up_both(); break; }
-          if (h == 0) {
-            float4* dst = reinterpret_cast<float4*>(g.nx_upart + ((size_t)nt * (size_t)g.Mp + (size_t)(row0 + lane)) * rn);
+            for (int c = 0; c < 4; ++c)
+              reinterpret_cast<float4*>(dst)[c] =
+                  make_float4(__uint_as_float(uv[4 * c]), __uint_as_float(uv[4 * c + 1]),
+                              __uint_as_float(uv[4 * c + 2]), __uint_as_float(uv[4 * c + 3]));
+          } else {
+            uint32_t uv[8];
+            tmem_ld_8cols(ua, uv);
+            tmem_ld_wait();
 #pragma unroll
-            for (int k4 = 0; k4 < kC_MaxR / 4; ++k4) {
-              if (4 * k4 < rn) {
-                const ulonglong2 o = xch[k4];
-                float a0, a1, a2, a3, b0, b1, b2, b3;
-                f2_unpack(u2[2 * k4], a0, a1); f2_unpack(u2[2 * k4 + 1], a2, a3);
-                f2_unpack(o.x, b0, b1); f2_unpack(o.y, b2, b3);
-                __stcg(dst + k4, make_float4(a0 + b0, a1 + b1, a2 + b2, a3 + b3));
-              }
-            }
+            for (int c = 0; c < 2; ++c)
+              reinterpret_cast<float4*>(dst)[c] =
+                  make_float4(__uint_as_float(uv[4 * c]), __uint_as_float(uv[4 * c + 1]),
+                              __uint_as_float(uv[4 * c + 2]), __uint_as_float(uv[4 * c + 3]));
           }
+          tc_fence_before();
         }
         continue;
       }
@@ -1765,12 +1773,16 @@ __global__ void __launch_bounds__(kSM_Threads, 1)
       auto stage_bytes = [&](int j) -> uint32_t {
         return j < cpk ? (uint32_t)(kTileCodes + 2048 + kSM_Tokens * 128 + 2048) : (uint32_t)(kLRTile + kSM_Tokens * 128);
       };
-      // the weights do not depend on the activation kernel: start them now
+      // the weights do not depend on the activation kernel: start them now,
+      // the first stages into shared memory and the rest of this CTA's slabs
+      // into L2
       const int first = steps < kSM_Stages ? steps : kSM_Stages;
       for (int j = 0; j < first; ++j) {
         mbar_arrive_expect_tx(&full_bar[j], stage_bytes(j));
         weight_part(j, smem + j * kSM_Stage);
       }
+      for (int j = first; j < cpk; ++j)
+        bulk_prefetch_l2(g.wtiles + ((size_t)nt * ksl + (size_t)(kq * cpk + j)) * kWTile, kWTile);
       griddep_wait();   // activation tiles and low-rank rows come from the activation kernel
       for (int j = 0; j < first; ++j) act_part(j, smem + j * kSM_Stage);
       int issued = first;
@@ -2400,7 +2412,7 @@ svdq_status device_ready() {
       d.ok = cudaFuncSetAttribute(dev::gemm_nvfp4_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   dev::kP_Smem) == cudaSuccess &&
              cudaFuncSetAttribute(dev::gemm_nvfp4_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  dev::kP_Smem) == cudaSuccess &&
+                                  dev::kC_Smem) == cudaSuccess &&
              cudaFuncSetAttribute(dev::gemm_nvfp4_small_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   dev::sm_smem(16)) == cudaSuccess &&
              cudaFuncSetAttribute(dev::gemm_nvfp4_small_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -2663,7 +2675,7 @@ svdq_status launch_gemm(const svdq_params* p, const void* blob_dev, int64_t M, v
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_pair_kernel<false>, g, tm_y);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_pair_kernel<false>, g, tm_y, tm_y);
     if (e != cudaSuccess) return cuda_fail(e, "gemm_nvfp4_pair_kernel launch");
     return launch_status("gemm_nvfp4_pair_kernel launch");
   }
@@ -2747,21 +2759,23 @@ svdq_status launch_gemm_chain(const svdq_params* p, const void* blob_dev, int64_
   g.nx_atiles = wsn + Wn.off_xq;
   g.nx_upart = reinterpret_cast<float*>(ws + C.off_extra);
   g.nx_r = rn;
-  g.nx_l1t = reinterpret_cast<const uint16_t*>(nblob + Bn.off_l1t);
-  const CUtensorMap unused_map{};   // the chained form writes no Y
+  CUtensorMap tm_l1n{};
+  if (rn > 0 && !make_map(&tm_l1n, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, nblob + Bn.off_l1t, (uint64_t)N, (uint64_t)rn,
+                          (uint64_t)N * 2, 64, (uint32_t)(rn / 2)))
+    return cuda_fail(cudaErrorInvalidValue, "tensor map encode (next layer L1)");
   const int tiles = (N / 256) * (int)(W.Mp / 256);
   const int pairs = std::max(1, std::min(tiles, num_sms() / 2));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
   cfg.blockDim = dim3(dev::kP_Threads);
-  cfg.dynamicSmemBytes = dev::kP_Smem;
+  cfg.dynamicSmemBytes = dev::kC_Smem;
   cfg.stream = stream;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_pair_kernel<true>, g, unused_map);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, dev::gemm_nvfp4_pair_kernel<true>, g, tm_l1n, tm_l1n);
   if (e != cudaSuccess) return cuda_fail(e, "gemm_nvfp4_pair_kernel (chained) launch");
   if (rn > 0) {
     const int lrw_n = lr_width(*pn);

@@ -1,16 +1,24 @@
-// Device half of libsvdq: the two kernels of svdq_linear and their launchers.
+// Device half of libsvdq: the kernels of svdq_linear and their launchers.
 //
-//   act_quant_kernel  (kernel 1)  reads X once: X^ = fp32(X) * inv_lambda,
-//       per-token dynamic 4-bit quantisation (NVFP4 blocks of 16 / INT4 groups
-//       of 64) and the low-rank down projection u = X^16 L1 on the tensor cores
+//   kernel 1 reads X once: X^ = fp32(X) * inv_lambda, per-token dynamic 4-bit
+//       quantisation (NVFP4 blocks of 16 / INT4 groups of 64) and the low-rank
+//       down projection u = X^16 L1 on the tensor cores
 //       ("AI图像生成4-bit量化技术解析与应用" 3.1: dynamic activation ranges;
-//       "SVDQuant是什么？" 技术原理: 16-bit low-rank branch).
-//   gemm_nvfp4_kernel / gemm_int4_kernel  (kernel 2)  the 4-bit GEMM
-//       Q(X^) Q(R) on tcgen05 with TMEM accumulators, fed by TMA; the low-rank
-//       up projection u L2 runs as extra bf16 K-steps into the same
-//       accumulator and the epilogue adds the bias and writes bf16 Y
+//       "SVDQuant是什么？" 技术原理: 16-bit low-rank branch):
+//     act_nvfp4_kernel  NVFP4 above 256 tokens: 128-token tiles, tcgen05;
+//     act_quant_kernel  INT4, and NVFP4 up to 256 tokens: 32-token groups,
+//                       mma.sync, K split over clusters (and the workspace).
+//   kernel 2, the 4-bit GEMM Q(X^) Q(R) on tcgen05 with TMEM accumulators;
+//       the low-rank up projection u L2 runs as extra bf16 K-steps into the
+//       same accumulator and the epilogue adds the bias and writes bf16 Y
 //       ("DeepCompressor…" SVDQuant section: the low-rank branch fused into
-//       the low-bit kernel so it costs no extra activation traffic).
+//       the low-bit kernel so it costs no extra activation traffic):
+//     gemm_nvfp4_pair_kernel<false>  NVFP4 above 128 tokens, CTA pairs;
+//     gemm_nvfp4_small_kernel<TOK>   NVFP4 up to 128 tokens, weight tile as A;
+//     gemm_int4_kernel               INT4 (E4M3-coded), group scales folded.
+//   chained layers: gemm_nvfp4_pair_kernel<true> writes the next layer's
+//       quantised input instead of Y, chain_u_kernel adds its per-tile
+//       partial down projections.
 //
 // Every wait on an mbarrier is bounded (about 1 s); a wait that gives up
 // records SVDQ_ERR_TIMEOUT in a device status word and the CTA winds down.

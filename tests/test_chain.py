@@ -152,3 +152,23 @@ def test_gpu_chain_flux_ffn(gpu):
     wl1 = synth.make_workload("flux_ffn_up_nvfp4")
     pp1, pp2, y1 = _pair(wl1, 3072, 32, seed=7)
     print(_check(pp1, pp2, wl1.X, y1))
+
+
+def test_chain_rejects_unsupported_pairs_before_any_launch():
+    """The chained call checks the pair of layers on the host and returns
+    before touching a device pointer (no GPU needed)."""
+    import torch
+    p1 = sv.params(512, 768, 32, "nvfp4", "bf16")
+    dummy = torch.zeros(1024, dtype=torch.uint8)
+    cases = [(sv.params(768, 512, 32, "int4", "bf16"), sv.ERR_UNSUPPORTED),
+             (sv.params(768, 512, 32, "nvfp4", "fp16"), sv.ERR_UNSUPPORTED),
+             (sv.params(768, 512, 48, "nvfp4", "bf16"), sv.ERR_UNSUPPORTED),
+             (sv.params(1024, 512, 32, "nvfp4", "bf16"), sv.ERR_INVALID_ARG)]
+    for p2, want in cases:
+        with pytest.raises(sv.SVDQError) as e:
+            sv.gemm_chain(p1, dummy, 300, p2, dummy, dummy, dummy)
+        assert e.value.status == want, (p2.K, p2.fmt, p2.act_dtype, p2.rank, e.value.status)
+    with pytest.raises(sv.SVDQError) as e:   # this layer INT4
+        sv.gemm_chain(sv.params(512, 768, 32, "int4", "bf16"), dummy, 300, sv.params(768, 512, 32, "nvfp4", "bf16"),
+                      dummy, dummy, dummy)
+    assert e.value.status == sv.ERR_UNSUPPORTED
